@@ -1,0 +1,384 @@
+"""Pins for the CPU oracle: each test ties one oracle function to something
+other than itself — a value the pages print, a closed form, an invariant, or
+brute force on a tiny input — chosen so that a dropped term, a wrong sign or
+index, or a transposed operand fails at least one of them.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from synthetic import ALPHA_GRID, CLIP_GRID, bf16_bits, bf16_to_f32, small_layer
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------- worked example
+def test_worked_example_16_levels():
+    """The tutorial's 16-level example: step 0.427, 0.21 -> 0, output error 21."""
+    g = json.load(open(os.path.join(GOLDEN, "worked_example_16level.json")))
+    grp = np.array([g["range_min"], g["range_max"], g["weight"]] + [0.0] * 125, np.float32)
+    q, d, z = oracle.quant_group(grp, oracle.ASYM)
+    assert round(float(d), 3) == g["step_printed"]
+    assert (q[0] - z) * d == pytest.approx(g["range_min"], abs=d / 2 * 1.0001)
+    assert (q[1] - z) * d == pytest.approx(g["range_max"], abs=d / 2 * 1.0001)
+    deq = (q[2] - z) * float(d)
+    assert deq == g["dequantised"]
+    err = abs(float(np.float32(g["weight"])) - deq)
+    assert err == pytest.approx(g["weight_error"], rel=1e-6)
+    assert err * g["activation"] == pytest.approx(g["output_error"], rel=1e-6)
+    # the symmetric grid over the same range also sends 0.21 to 0
+    qs, ds, zs = oracle.quant_group(grp, oracle.SYM)
+    assert qs[2] == 0 and zs == 0
+
+
+# ------------------------------------------------------------------ activation stats
+def test_act_stats_integer_closed_form():
+    """Integer-valued X: the fp64 sums are exact, so s_X = float32(S / N)."""
+    r = rng(1)
+    N, I = 300, 37                      # ragged: 3 chunks of 128 tokens, odd width
+    Xi = r.integers(-9, 10, size=(N, I))
+    Xi[:, 5] = 0                        # clamped column
+    Xi[:, 6] = -2                       # sign: |X| not X
+    got = oracle.act_stats(Xi.astype(np.float32), clamp_min=1e-4)
+    S = np.abs(Xi).sum(axis=0)          # exact integer sums
+    want = np.array([np.float32(float(Fraction(int(s), N))) for s in S])
+    want[5] = np.float32(1e-4)
+    assert np.array_equal(got, want)
+    assert got[6] == np.float32(2.0)
+
+
+def test_act_stats_fsum_within_one_ulp():
+    """Random fp32 X: agrees with the exactly rounded mean (math.fsum) to 1 ulp."""
+    r = rng(2)
+    N, I = 517, 24
+    X = (r.standard_normal((N, I)) * np.exp(r.uniform(-8, 8, size=(1, I)))).astype(np.float32)
+    got = oracle.act_stats(X)
+    for i in range(I):
+        ref = np.float32(math.fsum(abs(float(v)) for v in X[:, i]) / N)
+        assert abs(int(got[i].view(np.int32)) - int(ref.view(np.int32))) <= 1
+
+
+def test_act_stats_axis_and_bf16():
+    """Non-square bf16 input: reduced over tokens, one value per input channel."""
+    W, X = small_layer(8, 64, 200, seed=3)
+    s = oracle.act_stats(X)
+    assert s.shape == (64,)
+    Xf = bf16_to_f32(X).astype(np.float64)
+    assert np.allclose(s, np.abs(Xf).mean(axis=0), rtol=1e-6)
+    assert np.all(s >= np.float32(1e-4))
+
+
+# ------------------------------------------------------------------ scale vector
+def test_scale_vector_special_alphas():
+    r = rng(4)
+    sX = np.exp(r.uniform(-9, 4, size=257)).astype(np.float32)
+    s0 = oracle.scale_vector(sX, 0.0)
+    assert np.all(s0 == 1.0)                                   # alpha = 0: plain RTN
+    s1 = oracle.scale_vector(sX, 1.0)
+    assert s1.max() == 1.0 and s1[np.argmax(sX)] == 1.0
+    assert np.allclose(s1, sX.astype(np.float64) / sX.max(), rtol=2 ** -24)
+    sh = oracle.scale_vector(sX, 0.5)
+    ref = np.sqrt(sX.astype(np.float64) / float(sX.max()))
+    assert np.allclose(sh, ref, rtol=2 ** -23)
+
+
+def test_scale_vector_power_law_and_order():
+    r = rng(5)
+    sX = np.exp(r.uniform(-9, 4, size=300)).astype(np.float32)
+    for a in ALPHA_GRID[1:]:
+        s = oracle.scale_vector(sX, a)
+        assert s.max() == 1.0
+        lhs = np.log(s.astype(np.float64)) / a
+        rhs = np.log(sX.astype(np.float64)) - np.log(float(sX.max()))
+        assert np.allclose(lhs, rhs, rtol=1e-5, atol=1e-5 / a)
+        order = np.argsort(sX, kind="stable")
+        assert np.all(np.diff(s[order]) >= 0)
+
+
+# ------------------------------------------------------------------ quantizer
+def _brute_nearest(t, lo, hi):
+    """Nearest integer code to real t within [lo, hi], ties to the even code."""
+    best, bd = None, None
+    for c in range(lo, hi + 1):
+        dd = abs(Fraction(t) - c)
+        if bd is None or dd < bd or (dd == bd and c % 2 == 0):
+            best, bd = c, dd
+    return best
+
+
+def test_quant_group_ties_to_even():
+    g = np.array([7.0, 2.5, -1.5, 0.5, -0.5, 3.5, -6.5, 1.0], np.float32)
+    q, d, z = oracle.quant_group(g, oracle.SYM)
+    assert d == np.float32(1.0) and z == 0
+    assert list(q) == [7, 2, -2, 0, 0, 4, -6, 1]
+
+
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_quant_group_sym_brute_force(gs):
+    r = rng(6 + gs)
+    for trial in range(40):
+        w = (r.standard_normal(gs) * 10.0 ** r.uniform(-4, 1)).astype(np.float32)
+        q, d, z = oracle.quant_group(w, oracle.SYM)
+        a = np.abs(w).max()
+        assert d == np.float32(a) / np.float32(7.0)
+        assert z == 0
+        for k in range(gs):
+            t = np.float32(w[k]) / d            # the fp32 quotient the pages' Round sees
+            assert q[k] == _brute_nearest(float(t), -8, 7)
+            assert abs(float(w[k]) - q[k] * float(d)) <= float(d) / 2 * (1 + 1e-6)
+        assert abs(q[np.argmax(np.abs(w))]) == 7
+
+
+@pytest.mark.parametrize("gs", [32, 128])
+def test_quant_group_asym_brute_force(gs):
+    r = rng(7 + gs)
+    for trial in range(40):
+        w = (r.standard_normal(gs) * 0.05 + r.uniform(-0.02, 0.02)).astype(np.float32)
+        q, d, z = oracle.quant_group(w, oracle.ASYM)
+        mx, mn = w.max(), w.min()
+        assert d == (np.float32(mx) - np.float32(mn)) / np.float32(15.0)
+        assert 0 <= z <= 15
+        assert z == _brute_nearest(float(np.float32(-mn) / d), 0, 15)
+        for k in range(gs):
+            t = np.float32(w[k]) / d
+            assert q[k] == _brute_nearest(float(t) + z, 0, 15) or \
+                q[k] == min(max(_brute_nearest(float(t), -100, 100) + z, 0), 15)
+            assert abs(float(w[k]) - (q[k] - z) * float(d)) <= float(d) * (1 + 1e-6)
+        assert q[np.argmin(w)] <= 1 and q[np.argmax(w)] >= 14
+
+
+def test_quant_group_scale_invariance():
+    """Codes are invariant under w -> w * 2^k, Delta scales by 2^k."""
+    r = rng(8)
+    w = (r.standard_normal(128) * 0.03).astype(np.float32)
+    for qt in (oracle.SYM, oracle.ASYM):
+        q0, d0, z0 = oracle.quant_group(w, qt)
+        for k in (-7, -1, 3, 11):
+            q1, d1, z1 = oracle.quant_group(w * np.float32(2.0 ** k), qt)
+            assert np.array_equal(q0, q1) and z0 == z1
+            assert d1 == d0 * np.float32(2.0 ** k)
+
+
+def test_quant_group_degenerate_and_clip():
+    q, d, z = oracle.quant_group(np.zeros(64, np.float32), oracle.SYM)
+    assert d == 0 and np.all(q == 0)
+    q, d, z = oracle.quant_group(np.full(64, 0.3, np.float32), oracle.ASYM)
+    assert d == 0 and z == 0 and np.all(q == 0)
+    r = rng(9)
+    w = (r.standard_normal(128)).astype(np.float32)
+    q, d, z = oracle.quant_group(w, oracle.SYM, clip=0.5)
+    a = np.abs(w).max()
+    assert d == np.float32(np.float64(a) * 0.5) / np.float32(7.0)
+    big = np.abs(w) > 0.5 * a * 8.5 / 7
+    assert np.all(np.abs(q[big]) >= 7) and q.min() >= -8 and q.max() <= 7
+    assert np.any(q == -8) or np.any(q == 7)
+
+
+def test_rounding_error_statistics():
+    """Rounding error is ~U[0, 0.5] with mean 0.25 (paper summary, Method:
+    the empirical observations on Round)."""
+    r = rng(10)
+    errs = []
+    for _ in range(400):
+        w = r.uniform(-1, 1, 128).astype(np.float32)
+        w[0] = 1.0
+        q, d, z = oracle.quant_group(w, oracle.SYM)
+        errs.append(np.abs(w / d - q))
+    e = np.concatenate(errs)
+    assert e.max() <= 0.5 + 1e-6
+    assert abs(e.mean() - 0.25) < 0.01
+
+
+def test_salient_scaling_reduces_error():
+    """Scaling one non-extreme weight by s = 2 leaves Delta unchanged and halves
+    its expected error in original units (paper summary, Method: Err'/Err =
+    (Delta'/Delta)(1/s))."""
+    r = rng(11)
+    e1, e2 = [], []
+    for _ in range(3000):
+        w = r.uniform(-1, 1, 128).astype(np.float32)
+        w[0] = 1.0
+        w[1] = np.float32(r.uniform(-0.45, 0.45))
+        q, d, _ = oracle.quant_group(w, oracle.SYM)
+        e1.append(abs(float(w[1]) - q[1] * float(d)))
+        w2 = w.copy()
+        w2[1] *= np.float32(2.0)
+        q2, d2, _ = oracle.quant_group(w2, oracle.SYM)
+        assert d2 == d
+        e2.append(abs(q2[1] * float(d2) / 2.0 - float(w[1])))
+    ratio = np.mean(e2) / np.mean(e1)
+    assert 0.45 < ratio < 0.55
+
+
+# ------------------------------------------------------------------ loss
+def _lossless_layer(O, I, gs, seed):
+    """W with W*s exactly on the quantisation grid (s powers of two)."""
+    r = rng(seed)
+    s = (2.0 ** r.integers(-3, 1, size=I)).astype(np.float32)
+    s[0] = 1.0
+    codes = r.integers(-7, 8, size=(O, I))
+    codes[:, ::gs] = 7                               # every group reaches +-7
+    delta = (2.0 ** r.integers(-9, -5, size=(O, I // gs))).astype(np.float32)
+    W = (codes * np.repeat(delta, gs, axis=1) / s[None, :]).astype(np.float32)
+    return W, s, codes, delta
+
+
+def test_loss_zero_when_quantisation_is_exact():
+    """W X = (W s)(X / s): with Q exact on W*s, the objective is exactly 0."""
+    O, I, gs, N = 6, 256, 64, 40
+    W, s, codes, delta = _lossless_layer(O, I, gs, 12)
+    X = rng(13).integers(-3, 4, size=(N, I)).astype(np.float32)
+    c, d, z = oracle.quant_layer(W, s, gs, oracle.SYM)
+    assert np.array_equal(c, codes) and np.array_equal(d, delta)
+    tot, lr = oracle.layer_loss_rows(W, X, s, gs, c, d, z)
+    assert tot == 0.0 and np.all(lr == 0.0)
+
+
+def test_loss_single_perturbation_closed_form():
+    O, I, gs, N = 5, 128, 32, 33
+    W, s, codes, delta = _lossless_layer(O, I, gs, 14)
+    X = rng(15).integers(-5, 6, size=(N, I)).astype(np.float32)
+    c, d, z = oracle.quant_layer(W, s, gs, oracle.SYM)
+    o, k = 3, 77
+    c = c.copy()
+    c[o, k] += 1 if c[o, k] < 7 else -1
+    tot, lr = oracle.layer_loss_rows(W, X, s, gs, c, d, z)
+    e = float(d[o, k // gs]) / float(s[k])
+    want = e * e * float((X[:, k].astype(np.float64) ** 2).sum())
+    assert lr[o] == want and tot == want
+    assert np.all(np.delete(lr, o) == 0.0)
+
+
+def _brute_loss_rows(W, X, s, gs, c, d, z):
+    O, I = W.shape
+    out = []
+    for o in range(O):
+        acc = 0.0
+        dw = [(int(c[o, i]) - int(z[o, i // gs])) * float(d[o, i // gs]) / float(s[i])
+              - float(W[o, i]) for i in range(I)]
+        for n in range(X.shape[0]):
+            e = math.fsum(float(X[n, i]) * dw[i] for i in range(I))
+            acc += e * e
+        out.append(acc)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_loss_brute_force_tiny(qt):
+    W, X = small_layer(3, 64, 7, wdtype="f32", xdtype="f32", seed=16, n_outliers=2)
+    sX = oracle.act_stats(X)
+    s = oracle.scale_vector(sX, 0.35)
+    c, d, z = oracle.quant_layer(W, s, 32, qt)
+    tot, lr = oracle.layer_loss_rows(W, X, s, 32, c, d, z)
+    ref = _brute_loss_rows(W, X, s, 32, c, d, z)
+    assert np.allclose(lr, ref, rtol=1e-12, atol=0)
+
+
+def test_search_brute_force_argmin_and_invariants():
+    """Non-square tiny layer: the search's losses equal the brute-force losses
+    at each grid point, alpha* is their first minimiser, loss(alpha=0) is plain
+    RTN, and loss(clip = 1.0) equals loss(alpha*)."""
+    O, I, N, gs = 4, 96, 11, 32
+    W, X = small_layer(O, I, N, wdtype="f32", xdtype="f32", seed=17, n_outliers=3, outlier=30.0)
+    sX = oracle.act_stats(X)
+    alpha = ALPHA_GRID[::4]
+    res = oracle.search_layer(W, X, sX, gs, oracle.SYM, alpha, clip=CLIP_GRID[:4])
+    ref = []
+    for a in alpha:
+        s = oracle.scale_vector(sX, a)
+        c, d, z = oracle.quant_layer(W, s, gs, oracle.SYM)
+        ref.append(_brute_loss_rows(W, X, s, gs, c, d, z).sum() / (N * O))
+    assert np.allclose(res["loss"][:len(alpha)], ref, rtol=1e-12)
+    assert res["best_alpha"] == int(np.argmin(ref))
+    c, d, z = oracle.quant_layer(W, np.ones(I, np.float32), gs, oracle.SYM)
+    rtn = _brute_loss_rows(W, X, np.ones(I, np.float32), gs, c, d, z).sum() / (N * O)
+    assert res["loss"][0] == pytest.approx(rtn, rel=1e-12)
+    assert res["loss"][len(alpha)] == res["loss"][res["best_alpha"]]
+    assert res["best_clip"] == int(np.argmin(res["loss"][len(alpha):]))
+
+
+def test_search_first_minimum_on_ties():
+    """With X = 0 every loss is 0: the first grid point wins."""
+    W, _ = small_layer(4, 64, 8, seed=18)
+    X = np.zeros((8, 64), np.float32)
+    sX = oracle.act_stats(X)
+    res = oracle.search_layer(W, X, sX, 32, oracle.SYM, ALPHA_GRID[:5], clip=CLIP_GRID[:3])
+    assert np.all(res["loss"] == 0.0)
+    assert res["best_alpha"] == 0 and res["best_clip"] == 0
+
+
+def test_search_row_subset_matches_full():
+    W, X = small_layer(12, 64, 20, seed=19)
+    sX = oracle.act_stats(X)
+    full = oracle.search_layer(W, X, sX, 32, oracle.ASYM, ALPHA_GRID[:3])
+    rows = np.array([1, 5, 11])
+    sub = oracle.search_layer(W, X, sX, 32, oracle.ASYM, ALPHA_GRID[:3], rows=rows)
+    assert np.array_equal(sub["loss_row"], full["loss_row"][:, rows])
+
+
+# ------------------------------------------------------------------ pack
+@pytest.mark.parametrize("qt", [0, 1])
+def test_pack_layout(qt):
+    O, I, gs = 5, 640, 128               # 5 groups: a partly filled zero word
+    W, X = small_layer(O, I, 16, seed=20)
+    sX = oracle.act_stats(X)
+    p = oracle.pack_int4(W, sX, 0.45, 0.9, gs, qt)
+    s = oracle.scale_vector(sX, 0.45)
+    c, d, z = oracle.quant_layer(W, s, gs, qt, clip=0.9)
+    nib = np.stack([(p["qweight"] >> np.uint32(4 * k)) & np.uint32(15) for k in range(8)], axis=-1)
+    codes = nib.reshape(O, I).astype(np.int64)
+    assert np.array_equal(codes, c.astype(np.int64) + (8 if qt == 0 else 0))
+    assert np.array_equal(p["scales"], d.astype(np.float16).view(np.uint16))
+    assert np.array_equal(p["scales_f32"], d)
+    assert np.array_equal(p["s16"], s.astype(np.float16).view(np.uint16))
+    if qt == 1:
+        zn = np.stack([(p["zeros"] >> np.uint32(4 * k)) & np.uint32(15) for k in range(8)], axis=-1)
+        zn = zn.reshape(O, -1)
+        assert np.array_equal(zn[:, :I // gs], z.astype(np.uint32))
+        assert np.all(zn[:, I // gs:] == 0)
+    else:
+        assert p["zeros"] is None
+
+
+# ------------------------------------------------------------------ apply
+def test_apply_integer_closed_form():
+    """s = 1, Delta = 1, symmetric: y = x (codes - 8)^T exactly."""
+    r = rng(21)
+    M, I, O, gs = 3, 256, 7, 64
+    codes = r.integers(0, 16, size=(O, I)).astype(np.uint32)
+    qw = np.zeros((O, I // 8), np.uint32)
+    for k in range(8):
+        qw |= codes[:, k::8] << np.uint32(4 * k)
+    one16 = np.float16(1.0).view(np.uint16)
+    scales = np.full((O, I // gs), one16, np.uint16)
+    s16 = np.full(I, one16, np.uint16)
+    x = r.integers(-4, 5, size=(M, I))
+    y = oracle.linear_w4a16(x.astype(np.float32), qw, scales, None, s16, gs)
+    assert np.array_equal(y, (x @ (codes.astype(np.int64) - 8).T).astype(np.float64))
+
+
+def test_apply_matches_dense_dequant():
+    O, I, gs, M = 9, 384, 128, 4
+    W, X = small_layer(O, I, 32, seed=22)
+    sX = oracle.act_stats(X)
+    p = oracle.pack_int4(W, sX, 0.6, 1.0, gs, oracle.ASYM)
+    x = bf16_bits(rng(23).standard_normal((M, I)).astype(np.float32))
+    y = oracle.linear_w4a16(x, p["qweight"], p["scales"], p["zeros"], p["s16"], gs)
+    s = oracle.scale_vector(sX, 0.6)
+    c, d, z = oracle.quant_layer(W, s, gs, oracle.ASYM)
+    d16 = d.astype(np.float16).astype(np.float64)
+    deq = (c.astype(np.float64) - np.repeat(z.astype(np.float64), gs, axis=1)) * np.repeat(d16, gs, axis=1)
+    xs = bf16_to_f32(x).astype(np.float64) / s.astype(np.float16).astype(np.float64)[None, :]
+    assert np.allclose(y, xs @ deq.T, rtol=1e-12, atol=1e-12)
+    # and it approximates the unquantised layer
+    yf = bf16_to_f32(x).astype(np.float64) @ bf16_to_f32(W).astype(np.float64).T
+    assert np.linalg.norm(y - yf) < 0.2 * np.linalg.norm(yf)
