@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the AWQ per-layer scale search hot path on B200.
+
+One step = the whole path over one layer of the Llama-7B attention-projection
+workload (W 4096x4096 bf16, 4096 calibration tokens, symmetric INT4, group 128,
+20-point alpha grid): activation statistics -> fused grid search (fake
+quantisation, output-error contraction, loss reduction, argmin) -> INT4 packing
+at alpha* -> W4A16 apply at M = 1.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Metric: search TFLOP/s = grid * 2 * N * in * out per step / device time per
+step.  Inputs are resident in HBM when the timed region starts; three rotating
+copies of (W, X) (201 MB > 126 MB L2) keep each step's reads out of L2.  With N
+GPUs (torchrun, one process per GPU) every rank quantises its own layer
+(independent units, no data-path collective): weak scaling, time = max over
+ranks.  `--impl reference` times the CPU oracle on a bounded row sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "AWQ search TFLOP/s (grid×2·N·in·out), ms/layer, % BF16 peak; W4A16 GB/s"
+WORKLOAD_ID = 2
+LAYER = "attn_proj"
+GROUP = 128
+ROTATE = 3
+APPLY_M = 1
+
+# DRAM traffic of one search-kernel launch on this workload, from the ncu capture
+# summarised in profiles/search_kernel_attn_proj_4096.md, valid only for the
+# kernel source it was taken on (sha256 of csrc/k_search.cu, first 16 hex).
+SEARCH_TRAFFIC = {"source_sha": None, "bytes": None}
+
+
+def _env_int(k, d):
+    try:
+        return int(os.environ.get(k, d))
+    except ValueError:
+        return d
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def source_sha(path):
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[1]:
+                continue
+            rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        smax = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        loaded = [s for s in sm if s > 0.5 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[6 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import synthetic
+    import weight_only_quantization_awq_b200 as awq
+    from synthetic import ALPHA_GRID
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = synthetic.workload(WORKLOAD_ID)
+    L = wl.layers[0]
+    O, I, N, G = L.out, L.inp, wl.tokens, len(ALPHA_GRID)
+    flops_step = G * 2.0 * N * I * O
+
+    def to_dev(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    W_np = synthetic.layer_weights(WORKLOAD_ID, LAYER)
+    X_np = synthetic.layer_activations(WORKLOAD_ID, LAYER)
+    x_np = synthetic.apply_activations(APPLY_M, I)
+    Ws = [to_dev(W_np) for _ in range(ROTATE)]
+    Xs = [to_dev(X_np) for _ in range(ROTATE)]
+    xd = to_dev(x_np)
+    alphas = [float(a) for a in ALPHA_GRID]
+    awq.set_kernel_timing(True)
+    search_ms = []
+
+    def step(k, record):
+        Wd, Xd = Ws[k % ROTATE], Xs[k % ROTATE]
+        sX = awq.awq_act_stats(Xd)
+        res = awq.awq_search_layer(Wd, Xd, sX, GROUP, 4, "sym", alphas)
+        if record:
+            search_ms.append(awq.last_kernel_ms(awq.KT_SEARCH))
+        p = awq.awq_pack_int4(Wd, sX, alphas[res["best_alpha"]], 1.0, GROUP, "sym")
+        y = awq.awq_linear_w4a16(xd, p["qweight"], p["scales"], None, p["s16"], GROUP)
+        return res, p, y
+
+    for k in range(args.warmup):
+        step(k, False)
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for k in range(args.steps):
+        res, p, y = step(k, True)
+    ev1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = flops_step * args.steps * world / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API: pinned host inputs in, results out.
+    W_h = torch.from_numpy(W_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    X_h = torch.from_numpy(X_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Wd_e, Xd_e, xd_e = torch.empty_like(Ws[0]), torch.empty_like(Xs[0]), torch.empty_like(xd)
+    qh = torch.empty(p["qweight"].shape, dtype=torch.int32).pin_memory()
+    sh = torch.empty(p["scales"].shape, dtype=torch.float16).pin_memory()
+    s16h = torch.empty(p["s16"].shape, dtype=torch.float16).pin_memory()
+    yh = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        Wd_e.copy_(W_h, non_blocking=True)
+        Xd_e.copy_(X_h, non_blocking=True)
+        xd_e.copy_(x_h, non_blocking=True)
+        sX = awq.awq_act_stats(Xd_e)
+        r = awq.awq_search_layer(Wd_e, Xd_e, sX, GROUP, 4, "sym", alphas)
+        pk = awq.awq_pack_int4(Wd_e, sX, alphas[r["best_alpha"]], 1.0, GROUP, "sym")
+        yy = awq.awq_linear_w4a16(xd_e, pk["qweight"], pk["scales"], None, pk["s16"], GROUP)
+        qh.copy_(pk["qweight"], non_blocking=True)
+        sh.copy_(pk["scales"], non_blocking=True)
+        s16h.copy_(pk["s16"], non_blocking=True)
+        yh.copy_(yy, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    e2e_steps = max(1, min(args.steps, 50))
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = W_h.numel() * 2 + X_h.numel() * 2 + x_h.numel() * 2
+    d2h = qh.numel() * 4 + sh.numel() * 2 + s16h.numel() * 2 + yh.numel() * 2 + 8 * G + 4 * 8
+    e2e_value = flops_step * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    # ---- W4A16 apply at M = 1: rotating packed copies (> L2), one CUDA graph of launches.
+    n_copies = 16
+    packs = [awq.awq_pack_int4(Ws[0], sX_ := awq.awq_act_stats(Xs[0]), 0.5, 1.0, GROUP, "sym")
+             for _ in range(n_copies)]
+    ys = torch.empty((APPLY_M, O), dtype=torch.bfloat16, device=dev)
+    reps = 8
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    awq.set_kernel_timing(False)
+    with torch.cuda.stream(s):
+        for pk in packs:
+            awq.awq_linear_w4a16(xd, pk["qweight"], pk["scales"], None, pk["s16"], GROUP, out=ys)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            for pk in packs:
+                awq.awq_linear_w4a16(xd, pk["qweight"], pk["scales"], None, pk["s16"], GROUP,
+                                     out=ys)
+    g.replay()
+    torch.cuda.synchronize()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    g.replay()
+    a1.record()
+    torch.cuda.synchronize()
+    apply_us = a0.elapsed_time(a1) * 1e3 / (reps * n_copies)
+    apply_bytes = O * I // 2 + O * (I // GROUP) * 2 + I * 2 + APPLY_M * I * 2 + APPLY_M * O * 2
+    del g
+
+    pk_ = peaks()
+    search_kernel_ms = statistics.mean(search_ms) if search_ms else None
+    achieved = flops_step / (search_kernel_ms * 1e-3) / 1e12 if search_kernel_ms else None
+    sha = source_sha(os.path.join(ROOT, "weight_only_quantization_awq_b200", "csrc", "k_search.cu"))
+    traffic = SEARCH_TRAFFIC["bytes"] if SEARCH_TRAFFIC["source_sha"] == sha else None
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "out": O, "in": I, "tokens": N, "grid": G,
+                   "quant": "sym_int4", "group_size": GROUP, "apply_m": APPLY_M,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"},
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / e2e_steps, 4),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 11 * args.steps,
+        "clocks": clk,
+        "roofline": {"bound": "tensor", "kernel": "search_kernel",
+                     "achieved": round(achieved, 2) if achieved else None,
+                     "peak": pk_["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk_["bf16_tflops"], 4) if achieved else None,
+                     "peak_source": pk_["source"] + " burst bf16",
+                     "kernel_ms": round(search_kernel_ms, 4) if search_kernel_ms else None,
+                     "algorithmic_flops": flops_step,
+                     "traffic": traffic},
+        "ms_per_layer": round(ms_per_step, 4),
+        "pct_bf16_peak": round(100.0 * value / world / pk_["bf16_tflops"], 2),
+        "w4a16": {"m": APPLY_M, "us_per_launch": round(apply_us, 3),
+                  "gb_per_s": round(apply_bytes / (apply_us * 1e-6) / 1e9, 1),
+                  "frac_hbm": round(apply_bytes / (apply_us * 1e-6) / 1e9 / pk_["hbm_gbs"], 4),
+                  "bytes": apply_bytes, "timing": f"CUDA graph of {reps * n_copies} launches over {n_copies} packed copies"},
+    }
+    if rank == 0 and world == 1:
+        out["cpu_baseline"] = cpu_baseline(W_np, X_np)
+    if world > 1:
+        dist.barrier(device_ids=[local_rank])
+    return out
+
+
+# --------------------------------------------------------------- the oracle
+def _oracle_threads():
+    n = len(os.sched_getaffinity(0))
+    os.environ.setdefault("OMP_NUM_THREADS", str(n))
+    return int(os.environ["OMP_NUM_THREADS"])
+
+
+def oracle_step(W_np, X_np, rows):
+    """The oracle's pass of the path on a row sample: statistics over all of X,
+    the 20-point search evaluated on `rows`, packing of the whole layer."""
+    import oracle
+    from synthetic import ALPHA_GRID
+    sX = oracle.act_stats(X_np)
+    res = oracle.search_layer(W_np, X_np, sX, GROUP, 0, ALPHA_GRID, rows=rows)
+    oracle.pack_int4(W_np, sX, float(ALPHA_GRID[res["best_alpha"]]), 1.0, GROUP, 0)
+    return res
+
+
+def cpu_baseline(W_np, X_np, rows_per_core=16):
+    import numpy as np
+    cores = _oracle_threads()
+    O = W_np.shape[0]
+    R = min(O, rows_per_core * cores)
+    rows = np.arange(R, dtype=np.int64)
+    N, I = X_np.shape
+    t0 = time.perf_counter()
+    oracle_step(W_np, X_np, rows)
+    dt = time.perf_counter() - t0
+    flops = 20 * 2.0 * N * I * R
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"full statistics and packing, 20-point search on the first {R} of {O} rows "
+                      f"(grid*2*N*in*rows = {flops:.3e} flop)"}
+
+
+def run_reference(args):
+    import numpy as np
+    import synthetic
+    cores = _oracle_threads()
+    wl = synthetic.workload(WORKLOAD_ID)
+    L = wl.layers[0]
+    W_np = synthetic.layer_weights(WORKLOAD_ID, LAYER)
+    X_np = synthetic.layer_activations(WORKLOAD_ID, LAYER)
+    R = min(L.out, 4 * cores)
+    rows = np.arange(R, dtype=np.int64)
+    flops = 20 * 2.0 * wl.tokens * L.inp * R
+    for _ in range(args.warmup):
+        oracle_step(W_np, X_np, rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(W_np, X_np, rows)
+    dt = time.perf_counter() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = (f"per step: full statistics and packing, 20-point search on the first {R} of "
+              f"{L.out} rows")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "out": L.out, "in": L.inp, "tokens": wl.tokens,
+                       "grid": 20, "quant": "sym_int4", "group_size": GROUP},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local_rank = _env_int("LOCAL_RANK", 0)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

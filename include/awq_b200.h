@@ -1,0 +1,162 @@
+/*
+ * awq_b200.h — C ABI of the B200 (sm_100a) AWQ per-layer scale search.
+ *
+ * The operations follow the AWQ pages:
+ *   [AWQ-blog]  "AWQ: Activation-aware Weight Quantization ..." paper summary
+ *               (bg51717 blog), section Method: the quantizer
+ *               Q(w) = Delta*Round(w/Delta), the objective
+ *               L(s) = ||Q(W*s)(s^-1*X) - W X||, the grid s = s_X^alpha with
+ *               alpha* = argmin L, clipping of the enlarged weights.
+ *   [AWQ-guide] "AWQ 量化方案：激活感知的权重量化与工程实现全解析" (qwbw.cn),
+ *               section 三: act_norm = mean |X| over calibration tokens,
+ *               scale = act_norm^alpha / max, per-group Delta = max/7 with
+ *               codes clamped to [-8, 7], QuantLinear (INT4-packed weight,
+ *               per-group fp16 scales, per-channel scale applied to x).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major and live in device memory unless an argument says
+ *     "host".  W is [out, in], X is [N, in] (tokens x input channels).
+ *   - bf16 and fp16 values are passed as their 16-bit patterns (uint16_t).
+ *   - Device pointers must be 16-byte aligned (AWQ_ERR_ALIGN otherwise).
+ *   - The caller owns every buffer it passes.  The library allocates its own
+ *     temporary device workspace with stream-ordered allocation on `stream`
+ *     and frees it on the same stream before returning.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued on it; entry points return without synchronising unless noted.
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call returns AWQ_ERR_ARG / AWQ_ERR_ALIGN / AWQ_ERR_UNSUPPORTED
+ *     and enqueues nothing.  A failing CUDA call returns AWQ_ERR_CUDA (see
+ *     awq_last_error()).  In-kernel waits are bounded; a wait that gives up
+ *     is reported as AWQ_ERR_TIMEOUT by the next synchronising entry point.
+ *   - Supported: w_bit = 4; group_size in {32, 64, 128}; in % 64 == 0;
+ *     in % group_size == 0; any out >= 1 and N >= 1 (tails are masked).
+ */
+#ifndef AWQ_B200_H
+#define AWQ_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    AWQ_OK = 0,
+    AWQ_ERR_ARG = 1,          /* null pointer, non-positive size, bad enum    */
+    AWQ_ERR_ALIGN = 2,        /* device pointer not 16-byte aligned            */
+    AWQ_ERR_UNSUPPORTED = 3,  /* valid request outside the supported set      */
+    AWQ_ERR_CUDA = 4,         /* a CUDA runtime call failed                    */
+    AWQ_ERR_TIMEOUT = 5       /* a bounded in-kernel wait gave up              */
+} awq_status_t;
+
+typedef enum { AWQ_F32 = 0, AWQ_BF16 = 1 } awq_dtype_t;
+typedef enum { AWQ_SYM = 0, AWQ_ASYM = 1 } awq_quant_t;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int awq_version(void);
+
+/* Static string for a status code. */
+const char *awq_status_string(int status);
+
+/* Text of the last error seen by the calling host thread ("" if none). */
+const char *awq_last_error(void);
+
+/*
+ * awq_act_stats — per-input-channel activation statistic ([AWQ-guide] 三,
+ * step 1; [AWQ-blog] Method, s_X).
+ *     sX[i] = max(clamp_min, mean_n |X[n, i]|)
+ * X        : [N, in] device, fp32 or bf16 (x_dtype).
+ * sX       : [in] fp32 device, written.
+ * The mean accumulates in fp64: tokens are summed sequentially within chunks
+ * of 128 consecutive tokens and the chunk partials are added in ascending
+ * chunk order, then the fp64 mean is rounded once to fp32.
+ * Requires in % 8 == 0.  Asynchronous.
+ */
+awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in,
+                           float clamp_min, float *sX, void *stream);
+
+/*
+ * awq_search_layer — the AWQ grid search of one linear layer ([AWQ-blog]
+ * Method: s = s_X^alpha, alpha* = argmin_alpha L(s); clipping of the enlarged
+ * weights).  For every grid point k < n_alpha:
+ *     s_k[i]   = s_X[i]^alpha[k] / max_j s_X[j]^alpha[k]   (fp64 pow, fp32 result)
+ *     Q_k      = group-wise INT4 fake quantisation of W * s_k (quant, group_size)
+ *     loss[k]  = mean over (n, o) of ( sum_i X[n, i] * (Q_k[o, i] / s_k[i] - W[o, i]) )^2
+ * best_alpha = first k with the minimal loss.  Then, if n_clip > 0, with s fixed
+ * at alpha[best_alpha], the same loss for each clip ratio clip[j] (the group
+ * bounds are multiplied by clip[j] before Delta is formed; values beyond them
+ * saturate), stored at loss[n_alpha + j]; best_clip = first minimiser.
+ * Quantizers: AWQ_SYM  Delta = max|w|/7, q = clamp(rint(w/Delta), -8, 7);
+ *             AWQ_ASYM Delta = (max w - min w)/15, z = clamp(rint(-min/Delta), 0, 15),
+ *                      q = clamp(rint(w/Delta) + z, 0, 15), value (q - z)*Delta.
+ * W         : [out, in] device, fp32 or bf16 (w_dtype).
+ * X         : [N, in] device, fp32 or bf16 (x_dtype); fp32 X is rounded to bf16
+ *             for the tensor-core contraction.
+ * sX        : [in] fp32 device (from awq_act_stats).
+ * alpha     : [n_alpha] host, 1 <= n_alpha <= 64, each in [0, 1].
+ * clip      : [n_clip] host or NULL, 0 <= n_clip <= 64, each in (0, 1].
+ * loss      : [n_alpha + n_clip] host fp64, written.
+ * loss_row  : optional [n_alpha + n_clip][out] fp32 device: per-row sums of
+ *             squared output error (not divided by N).
+ * best_alpha, best_clip : host, written (best_clip = -1 when n_clip == 0).
+ * Synchronises `stream` (the losses are returned on the host).
+ */
+awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t in,
+                              const void *X, int x_dtype, int64_t N,
+                              const float *sX, int group_size, int w_bit, int quant,
+                              const double *alpha, int n_alpha,
+                              const double *clip, int n_clip,
+                              double *loss, float *loss_row,
+                              int *best_alpha, int *best_clip, void *stream);
+
+/*
+ * awq_pack_int4 — final quantisation at (alpha, clip) and INT4 packing
+ * ([AWQ-guide] 三, step 4 and QuantLinear storage).  Bit-exact IEEE fp32:
+ * W' = W*s (one multiply), Delta = bound/7 or range/15 (correctly rounded
+ * divide), q from rint of the correctly rounded quotient W'/Delta.
+ * qweight    : [out][in/8] u32 device: nibble k (bits 4k..4k+3) of word w holds
+ *              column 8w+k; symmetric codes are stored as q+8, asymmetric as q.
+ * scales     : [out][in/group_size] fp16 bits device: Delta rounded to nearest even.
+ * zeros      : [out][ceil(in/group_size/8)] u32 device, nibble k of word w holds
+ *              z of group 8w+k; required for AWQ_ASYM, must be NULL for AWQ_SYM.
+ * s16        : [in] fp16 bits device: the per-channel scale s.
+ * scales_f32 : optional [out][in/group_size] fp32 device: Delta as computed.
+ * Asynchronous.
+ */
+awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in,
+                           const float *sX, double alpha, double clip,
+                           int group_size, int quant,
+                           uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
+                           uint16_t *s16, float *scales_f32, void *stream);
+
+/*
+ * awq_linear_w4a16 — the W4A16 layer that applies the result ([AWQ-guide] 三,
+ * QuantLinear.forward: x rescaled by the per-channel scale, weight dequantised
+ * per group, linear):
+ *     y[m, o] = sum_i (x[m, i] / s16[i]) * (code[o, i] - z[o, i/gs]) * scales[o, i/gs]
+ * with z = 8 when zeros == NULL (symmetric storage).  fp32 accumulation.
+ * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.
+ * Storage arguments as produced by awq_pack_int4.  Asynchronous.
+ */
+awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
+                              const uint32_t *qweight, const uint16_t *scales,
+                              const uint32_t *zeros, const uint16_t *s16,
+                              int group_size, uint16_t *y, void *stream);
+
+/*
+ * Kernel timing (instrumentation, off by default).  When enabled, each entry
+ * point brackets its main kernel launch(es) with CUDA events on `stream`;
+ * awq_last_kernel_ms(kind) returns the device time of that kernel in the last
+ * call of the calling host thread (summed over the two search phases), waiting
+ * for the end event if needed.  Returns a negative value if nothing was timed.
+ *   kind: 0 = activation statistics (both kernels), 1 = fused search kernel,
+ *         2 = pack kernel, 3 = W4A16 apply kernel.
+ */
+void awq_set_kernel_timing(int enable);
+double awq_last_kernel_ms(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AWQ_B200_H */

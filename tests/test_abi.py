@@ -1,0 +1,107 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+entry point the public header declares, and rejects invalid calls on the host
+with the documented status before any CUDA work is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "awq_b200.h")
+
+awq = pytest.importorskip("weight_only_quantization_awq_b200")
+lib = awq.lib
+
+OK, ARG, ALIGN, UNSUP = 0, 1, 2, 3
+FAKE = 0x10000          # a 16-byte aligned address that is never dereferenced
+NULL = None
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:awq_status_t|int|void|double|const char \*)\s*\*?(awq_\w+)\s*\(",
+                                 text, re.M)))
+
+
+def test_header_symbols_exported():
+    syms = header_symbols()
+    assert {"awq_act_stats", "awq_search_layer", "awq_pack_int4", "awq_linear_w4a16"} <= set(syms)
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) <= set(awq.EXPORTS)
+
+
+def test_version_and_status_strings():
+    assert lib.awq_version() >= 100
+    names = [lib.awq_status_string(k).decode() for k in range(6)]
+    assert names == ["AWQ_OK", "AWQ_ERR_ARG", "AWQ_ERR_ALIGN", "AWQ_ERR_UNSUPPORTED",
+                     "AWQ_ERR_CUDA", "AWQ_ERR_TIMEOUT"]
+
+
+def _search(**kw):
+    a = (ctypes.c_double * 20)(*[k / 20 for k in range(20)])
+    c = (ctypes.c_double * 3)(1.0, 0.9, 0.8)
+    loss = (ctypes.c_double * 23)()
+    ba, bc = ctypes.c_int(), ctypes.c_int()
+    args = dict(W=FAKE, wdt=1, out=256, inp=512, X=FAKE, xdt=1, N=1024, sX=FAKE, gs=128, wbit=4,
+                quant=0, alpha=a, na=20, clip=c, nc=3, loss=loss, lrow=NULL,
+                ba=ctypes.byref(ba), bc=ctypes.byref(bc), st=NULL)
+    args.update(kw)
+    return lib.awq_search_layer(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(W=NULL), ARG), (dict(wdt=7), ARG), (dict(out=0), ARG), (dict(quant=2), ARG),
+    (dict(gs=96), UNSUP), (dict(gs=256), UNSUP), (dict(inp=520), UNSUP), (dict(wbit=3), UNSUP),
+    (dict(W=FAKE + 8), ALIGN), (dict(X=FAKE + 4), ALIGN), (dict(na=0), ARG), (dict(na=65), ARG),
+    (dict(nc=-1), ARG), (dict(clip=NULL), ARG), (dict(N=0), ARG), (dict(loss=NULL), ARG),
+    (dict(alpha=(ctypes.c_double * 20)(*([0.5] * 19 + [1.5]))), ARG),
+    (dict(clip=(ctypes.c_double * 3)(1.0, 0.0, 0.5)), ARG),
+])
+def test_search_rejects_on_host(kw, status):
+    assert _search(**kw) == status
+    assert lib.awq_last_error().decode() != ""
+
+
+def test_act_stats_rejects_on_host():
+    f = lib.awq_act_stats
+    assert f(NULL, 1, 16, 64, ctypes.c_float(1e-4), FAKE, NULL) == ARG
+    assert f(FAKE, 3, 16, 64, ctypes.c_float(1e-4), FAKE, NULL) == ARG
+    assert f(FAKE, 1, 0, 64, ctypes.c_float(1e-4), FAKE, NULL) == ARG
+    assert f(FAKE, 1, 16, 12, ctypes.c_float(1e-4), FAKE, NULL) == UNSUP
+    assert f(FAKE + 2, 1, 16, 64, ctypes.c_float(1e-4), FAKE, NULL) == ALIGN
+    assert f(FAKE, 1, 16, 64, ctypes.c_float(-1.0), FAKE, NULL) == ARG
+
+
+def test_pack_rejects_on_host():
+    f = lib.awq_pack_int4
+    base = [FAKE, 1, 128, 256, FAKE, ctypes.c_double(0.5), ctypes.c_double(1.0), 128, 0,
+            FAKE, FAKE, NULL, FAKE, NULL, NULL]
+    def call(kw):
+        a = list(base)
+        for k, v in kw.items():
+            a[k] = v
+        return f(*a)
+    assert call({11: FAKE}) == ARG               # zeros given for symmetric storage
+    assert call({8: 1}) == ARG                   # asymmetric without zeros
+    assert call({5: ctypes.c_double(-0.1)}) == ARG
+    assert call({6: ctypes.c_double(0.0)}) == ARG
+    assert call({7: 48}) == UNSUP
+    assert call({9: FAKE + 4}) == ALIGN
+    assert call({4: NULL}) == ARG
+
+
+def test_linear_rejects_on_host():
+    f = lib.awq_linear_w4a16
+    base = [FAKE, 1, 4096, 4096, FAKE, FAKE, NULL, FAKE, 128, FAKE, NULL]
+    def call(kw):
+        a = list(base)
+        for k, v in kw.items():
+            a[k] = v
+        return f(*a)
+    assert call({0: NULL}) == ARG
+    assert call({1: 0}) == ARG
+    assert call({2: 100}) == UNSUP
+    assert call({8: 16}) == UNSUP
+    assert call({0: FAKE + 2}) == ALIGN

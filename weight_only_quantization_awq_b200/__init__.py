@@ -1,0 +1,199 @@
+"""B200 (sm_100a) AWQ per-layer scale search — Python binding.
+
+Thin ctypes marshalling over libawq_b200.so (C ABI in include/awq_b200.h):
+torch tensors supply device memory and the current CUDA stream, every step of
+the computation runs in the library's kernels.  The functions carry the C
+names:
+
+    awq_act_stats(X)                         -> s_X = mean |X| per input channel
+    awq_search_layer(W, X, sX, ...)          -> losses over the alpha (and clip) grid, argmin
+    awq_pack_int4(W, sX, alpha, clip, ...)   -> packed INT4 codes, fp16 scales, zeros, s
+    awq_linear_w4a16(x, packed...)           -> y = (x / s) @ dequant(W)^T
+
+Importing raises ImportError when the compiled library is missing; there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libawq_b200.so")
+
+AWQ_F32, AWQ_BF16 = 0, 1
+AWQ_SYM, AWQ_ASYM = 0, 1
+
+ALPHA_GRID_20 = tuple(k / 20.0 for k in range(20))
+
+
+class AwqError(RuntimeError):
+    """A library call returned a non-OK status."""
+
+    def __init__(self, fn: str, status: int, status_name: str, detail: str):
+        super().__init__(f"{fn}: {status_name}: {detail}")
+        self.status = status
+        self.status_name = status_name
+
+
+def _load_library() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python weight_only_quantization_awq_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, L, F, D = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                     ctypes.c_double)
+    lib.awq_version.restype = I
+    lib.awq_status_string.restype = ctypes.c_char_p
+    lib.awq_status_string.argtypes = [I]
+    lib.awq_last_error.restype = ctypes.c_char_p
+    lib.awq_act_stats.restype = I
+    lib.awq_act_stats.argtypes = [P, I, L, L, F, P, P]
+    lib.awq_search_layer.restype = I
+    lib.awq_search_layer.argtypes = [P, I, L, L, P, I, L, P, I, I, I, P, I, P, I, P, P, P, P, P]
+    lib.awq_pack_int4.restype = I
+    lib.awq_pack_int4.argtypes = [P, I, L, L, P, D, D, I, I, P, P, P, P, P, P]
+    lib.awq_linear_w4a16.restype = I
+    lib.awq_linear_w4a16.argtypes = [P, L, L, L, P, P, P, P, I, P, P]
+    lib.awq_set_kernel_timing.restype = None
+    lib.awq_set_kernel_timing.argtypes = [I]
+    lib.awq_last_kernel_ms.restype = D
+    lib.awq_last_kernel_ms.argtypes = [I]
+    return lib
+
+
+lib = _load_library()
+
+EXPORTS = ("awq_version", "awq_status_string", "awq_last_error", "awq_act_stats",
+           "awq_search_layer", "awq_pack_int4", "awq_linear_w4a16", "awq_set_kernel_timing",
+           "awq_last_kernel_ms")
+
+KT_STATS, KT_SEARCH, KT_PACK, KT_APPLY = 0, 1, 2, 3
+
+
+def set_kernel_timing(enable: bool) -> None:
+    """Bracket each entry point's main kernel(s) with CUDA events (thread-local)."""
+    lib.awq_set_kernel_timing(1 if enable else 0)
+
+
+def last_kernel_ms(kind: int) -> float:
+    """Device milliseconds of that kernel in the calling thread's last call (< 0: none)."""
+    return float(lib.awq_last_kernel_ms(kind))
+
+
+def _check(fn: str, status: int) -> None:
+    if status != 0:
+        raise AwqError(fn, status, lib.awq_status_string(status).decode(),
+                       lib.awq_last_error().decode())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return AWQ_F32
+    if t.dtype == torch.bfloat16:
+        return AWQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _quant_code(quant) -> int:
+    if quant in (AWQ_SYM, "sym", "symmetric"):
+        return AWQ_SYM
+    if quant in (AWQ_ASYM, "asym", "asymmetric"):
+        return AWQ_ASYM
+    raise ValueError(f"quant must be 'sym' or 'asym', got {quant!r}")
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def awq_act_stats(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.Tensor | None = None):
+    """s_X[i] = max(clamp_min, mean_n |X[n, i]|) for X [N, in] (fp32 or bf16)."""
+    _dev(X, "X")
+    N, inp = X.shape
+    if out is None:
+        out = torch.empty(inp, dtype=torch.float32, device=X.device)
+    _check("awq_act_stats", lib.awq_act_stats(X.data_ptr(), _dtype_code(X), N, inp,
+                                              float(clamp_min), out.data_ptr(), _stream(X)))
+    return out
+
+
+def awq_search_layer(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, group_size: int = 128,
+                     w_bit: int = 4, quant="sym", alpha=ALPHA_GRID_20, clip=None,
+                     loss_row: bool = False):
+    """Grid search of one layer.  Returns dict(loss: np.ndarray [G + C] fp64,
+    loss_row: tensor [G + C, out] fp32 or None, best_alpha, best_clip)."""
+    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
+    out_f, inp = W.shape
+    N = X.shape[0]
+    if X.shape[1] != inp or sX.numel() != inp:
+        raise ValueError("W, X and sX disagree on the input width")
+    a = np.ascontiguousarray(np.asarray(alpha, dtype=np.float64))
+    c = np.ascontiguousarray(np.asarray([] if clip is None else clip, dtype=np.float64))
+    loss = np.empty(a.size + c.size, np.float64)
+    lr = (torch.empty((a.size + c.size, out_f), dtype=torch.float32, device=W.device)
+          if loss_row else None)
+    ba, bc = ctypes.c_int(), ctypes.c_int()
+    st = lib.awq_search_layer(
+        W.data_ptr(), _dtype_code(W), out_f, inp, X.data_ptr(), _dtype_code(X), N, sX.data_ptr(),
+        group_size, w_bit, _quant_code(quant), a.ctypes.data, a.size,
+        c.ctypes.data if c.size else None, c.size, loss.ctypes.data,
+        lr.data_ptr() if lr is not None else None, ctypes.byref(ba), ctypes.byref(bc), _stream(W))
+    _check("awq_search_layer", st)
+    return {"loss": loss, "loss_row": lr, "best_alpha": ba.value, "best_clip": bc.value}
+
+
+def awq_pack_int4(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float = 1.0,
+                  group_size: int = 128, quant="sym", scales_f32: bool = False):
+    """Packed storage at (alpha, clip): dict(qweight int32 [out, in/8] (u32 bits),
+    scales fp16 [out, in/gs], zeros int32 [out, ceil(in/gs/8)] or None,
+    s16 fp16 [in], scales_f32 fp32 or None)."""
+    _dev(W, "W"), _dev(sX, "sX")
+    out_f, inp = W.shape
+    q = _quant_code(quant)
+    nG = inp // group_size
+    dev = W.device
+    qweight = torch.empty((out_f, inp // 8), dtype=torch.int32, device=dev)
+    scales = torch.empty((out_f, nG), dtype=torch.float16, device=dev)
+    zeros = (torch.empty((out_f, (nG + 7) // 8), dtype=torch.int32, device=dev)
+             if q == AWQ_ASYM else None)
+    s16 = torch.empty(inp, dtype=torch.float16, device=dev)
+    sf = torch.empty((out_f, nG), dtype=torch.float32, device=dev) if scales_f32 else None
+    st = lib.awq_pack_int4(
+        W.data_ptr(), _dtype_code(W), out_f, inp, sX.data_ptr(), float(alpha), float(clip),
+        group_size, q, qweight.data_ptr(), scales.data_ptr(),
+        zeros.data_ptr() if zeros is not None else None, s16.data_ptr(),
+        sf.data_ptr() if sf is not None else None, _stream(W))
+    _check("awq_pack_int4", st)
+    return {"qweight": qweight, "scales": scales, "zeros": zeros, "s16": s16, "scales_f32": sf,
+            "group_size": group_size}
+
+
+def awq_linear_w4a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                     zeros: torch.Tensor | None, s16: torch.Tensor, group_size: int = 128,
+                     out: torch.Tensor | None = None):
+    """y [M, out] bf16 = (x / s16) @ dequant(qweight, scales, zeros)^T for bf16 x [M, in]."""
+    _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales"), _dev(s16, "s16")
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    M, inp = x.shape
+    out_f = qweight.shape[0]
+    if out is None:
+        out = torch.empty((M, out_f), dtype=torch.bfloat16, device=x.device)
+    st = lib.awq_linear_w4a16(
+        x.data_ptr(), M, inp, out_f, qweight.data_ptr(), scales.data_ptr(),
+        zeros.data_ptr() if zeros is not None else None, s16.data_ptr(), group_size,
+        out.data_ptr(), _stream(x))
+    _check("awq_linear_w4a16", st)
+    return out

@@ -1,0 +1,422 @@
+// C ABI of the library (declared in include/awq_b200.h).  This layer checks
+// arguments on the host, sizes and allocates the temporary device workspace
+// with stream-ordered allocation, builds the TMA descriptor of the
+// calibration activations, and enqueues the kernels.  No arithmetic of the
+// method runs here: every step is a kernel.
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/awq_b200.h"
+#include "awq_internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+awq_status_t fail(awq_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+awq_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(AWQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define AWQ_CUDA(call)                                          \
+    do {                                                        \
+        cudaError_t e_ = (call);                                \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call);     \
+    } while (0)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device facts and one-time set-up (SM count; the default memory pool keeps
+// freed blocks cached so stream-ordered workspace allocation is cheap).
+struct DeviceInfo {
+    int sms = 0;
+    bool ready = false;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+awq_status_t device_info(int *sms) {
+    int dev = 0;
+    AWQ_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(AWQ_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        AWQ_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        cudaMemPool_t pool;
+        AWQ_CUDA(cudaDeviceGetDefaultMemPool(&pool, dev));
+        uint64_t thr = UINT64_MAX;
+        AWQ_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr));
+        d.ready = true;
+    }
+    *sms = d.sms;
+    return AWQ_OK;
+}
+
+// Temporary device workspace: one stream-ordered allocation per call, carved
+// into 256-byte aligned pieces, freed on the same stream when the call ends.
+struct Workspace {
+    cudaStream_t st;
+    char *base = nullptr;
+    size_t size = 0, used = 0;
+    explicit Workspace(cudaStream_t s) : st(s) {}
+    ~Workspace() {
+        if (base) cudaFreeAsync(base, st);
+    }
+    static size_t up(size_t b) { return (b + 255) & ~static_cast<size_t>(255); }
+    awq_status_t reserve(size_t bytes) {
+        size = bytes;
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void **>(&base), bytes, st);
+        if (e != cudaSuccess) {
+            base = nullptr;
+            return cuda_fail(e, "cudaMallocAsync(workspace)");
+        }
+        return AWQ_OK;
+    }
+    template <typename T>
+    T *take(size_t count) {
+        T *p = reinterpret_cast<T *>(base + used);
+        used += up(count * sizeof(T));
+        return p;
+    }
+};
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of the fp16 copy of X [N, I]: boxes of 64 channels x 256 tokens, 128-byte
+// swizzle (the K-major layout the MMA descriptors describe), zero fill out of
+// bounds so ragged token tails contribute nothing.
+awq_status_t make_x_map(CUtensorMap *map, const void *X, int64_t N, int64_t I) {
+    auto enc = get_encode();
+    if (!enc) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(I) * 2};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(awq::SLAB_K), static_cast<cuuint32_t>(awq::SUB_N)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return AWQ_OK;
+}
+
+bool valid_dtype(int d) { return d == AWQ_F32 || d == AWQ_BF16; }
+
+// Optional CUDA-event timing of the main kernels (see awq_set_kernel_timing).
+constexpr int KT_KINDS = 4;
+thread_local bool t_timing = false;
+struct KTimer {
+    cudaEvent_t beg[2] = {nullptr, nullptr}, end[2] = {nullptr, nullptr};
+    int n = 0;
+};
+thread_local KTimer t_kt[KT_KINDS];
+
+void kt_reset(int kind) {
+    KTimer &k = t_kt[kind];
+    for (int i = 0; i < 2; ++i) {
+        if (k.beg[i]) cudaEventDestroy(k.beg[i]);
+        if (k.end[i]) cudaEventDestroy(k.end[i]);
+        k.beg[i] = k.end[i] = nullptr;
+    }
+    k.n = 0;
+}
+
+void kt_begin(int kind, cudaStream_t st) {
+    if (!t_timing) return;
+    KTimer &k = t_kt[kind];
+    if (k.n >= 2) return;
+    cudaEventCreate(&k.beg[k.n]);
+    cudaEventCreate(&k.end[k.n]);
+    cudaEventRecord(k.beg[k.n], st);
+}
+
+void kt_end(int kind, cudaStream_t st) {
+    if (!t_timing) return;
+    KTimer &k = t_kt[kind];
+    if (k.n >= 2 || !k.end[k.n]) return;
+    cudaEventRecord(k.end[k.n], st);
+    ++k.n;
+}
+
+awq_status_t check_layer(const void *W, int w_dtype, int64_t out, int64_t in, int group_size,
+                         int quant) {
+    if (!W) return fail(AWQ_ERR_ARG, "W is NULL");
+    if (!valid_dtype(w_dtype)) return fail(AWQ_ERR_ARG, "bad w_dtype %d", w_dtype);
+    if (out < 1 || in < 1) return fail(AWQ_ERR_ARG, "bad shape out=%lld in=%lld", (long long)out, (long long)in);
+    if (quant != AWQ_SYM && quant != AWQ_ASYM) return fail(AWQ_ERR_ARG, "bad quant %d", quant);
+    if (group_size != 32 && group_size != 64 && group_size != 128)
+        return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
+    if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 64", (long long)in);
+    if (in > (1 << 20) || out > (1 << 24)) return fail(AWQ_ERR_UNSUPPORTED, "layer too large");
+    if (!aligned16(W)) return fail(AWQ_ERR_ALIGN, "W not 16-byte aligned");
+    return AWQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int awq_version(void) { return 100; }
+
+const char *awq_status_string(int status) {
+    switch (status) {
+        case AWQ_OK: return "AWQ_OK";
+        case AWQ_ERR_ARG: return "AWQ_ERR_ARG";
+        case AWQ_ERR_ALIGN: return "AWQ_ERR_ALIGN";
+        case AWQ_ERR_UNSUPPORTED: return "AWQ_ERR_UNSUPPORTED";
+        case AWQ_ERR_CUDA: return "AWQ_ERR_CUDA";
+        case AWQ_ERR_TIMEOUT: return "AWQ_ERR_TIMEOUT";
+        default: return "AWQ_ERR_UNKNOWN";
+    }
+}
+
+const char *awq_last_error(void) { return g_last_error.c_str(); }
+
+void awq_set_kernel_timing(int enable) {
+    t_timing = enable != 0;
+    for (int k = 0; k < KT_KINDS; ++k) kt_reset(k);
+}
+
+double awq_last_kernel_ms(int kind) {
+    if (kind < 0 || kind >= KT_KINDS) return -1.0;
+    KTimer &k = t_kt[kind];
+    if (k.n == 0) return -1.0;
+    double total = 0.0;
+    for (int i = 0; i < k.n; ++i) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(k.end[i]) != cudaSuccess) return -1.0;
+        if (cudaEventElapsedTime(&ms, k.beg[i], k.end[i]) != cudaSuccess) return -1.0;
+        total += ms;
+    }
+    return total;
+}
+
+awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in, float clamp_min,
+                           float *sX, void *stream) {
+    g_last_error.clear();
+    if (!X || !sX) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
+    if (N < 1 || in < 1) return fail(AWQ_ERR_ARG, "bad shape N=%lld in=%lld", (long long)N, (long long)in);
+    if (in % 8 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 8", (long long)in);
+    if (N > (int64_t(1) << 31) / 1) return fail(AWQ_ERR_UNSUPPORTED, "N too large");
+    if (!(clamp_min >= 0.0f)) return fail(AWQ_ERR_ARG, "clamp_min must be >= 0");
+    if (!aligned16(X) || !aligned16(sX)) return fail(AWQ_ERR_ALIGN, "X/sX not 16-byte aligned");
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t n_chunks = (N + awq::STATS_CHUNK - 1) / awq::STATS_CHUNK;
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(double) * n_chunks * in))) return s;
+    double *part = ws.take<double>(n_chunks * in);
+    kt_reset(0);
+    kt_begin(0, st);
+    AWQ_CUDA(awq::launch_stats_partial(X, x_dtype == AWQ_BF16, N, in, part, st));
+    AWQ_CUDA(awq::launch_stats_final(part, N, in, clamp_min, sX, st));
+    kt_end(0, st);
+    return AWQ_OK;
+}
+
+awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t in, const void *X,
+                              int x_dtype, int64_t N, const float *sX, int group_size, int w_bit,
+                              int quant, const double *alpha, int n_alpha, const double *clip,
+                              int n_clip, double *loss, float *loss_row, int *best_alpha,
+                              int *best_clip, void *stream) {
+    g_last_error.clear();
+    if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
+    if (w_bit != 4) return fail(AWQ_ERR_UNSUPPORTED, "w_bit %d (only 4)", w_bit);
+    if (!X || !sX || !alpha || !loss || !best_alpha || !best_clip)
+        return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
+    if (N < 1 || N > (int64_t(1) << 30)) return fail(AWQ_ERR_ARG, "bad N=%lld", (long long)N);
+    if (n_alpha < 1 || n_alpha > awq::MAX_GRID) return fail(AWQ_ERR_ARG, "n_alpha=%d", n_alpha);
+    if (n_clip < 0 || n_clip > awq::MAX_GRID || (n_clip > 0 && !clip))
+        return fail(AWQ_ERR_ARG, "n_clip=%d", n_clip);
+    for (int k = 0; k < n_alpha; ++k)
+        if (!(alpha[k] >= 0.0 && alpha[k] <= 1.0)) return fail(AWQ_ERR_ARG, "alpha[%d] out of [0,1]", k);
+    for (int k = 0; k < n_clip; ++k)
+        if (!(clip[k] > 0.0 && clip[k] <= 1.0)) return fail(AWQ_ERR_ARG, "clip[%d] out of (0,1]", k);
+    if (!aligned16(X) || !aligned16(sX) || (loss_row && !aligned16(loss_row)))
+        return fail(AWQ_ERR_ALIGN, "device pointer not 16-byte aligned");
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const int G = n_alpha > n_clip ? n_alpha : n_clip;
+    const int64_t nG = in / group_size;
+    const int64_t TB = (N + awq::TILE_N - 1) / awq::TILE_N;
+    const int Gtot = n_alpha + n_clip;
+    size_t bytes = 0;
+    bytes += Workspace::up(sizeof(uint16_t) * N * in);
+    bytes += 2 * Workspace::up(sizeof(float) * G * in);
+    bytes += Workspace::up(sizeof(float4) * G * out * nG);
+    bytes += Workspace::up(sizeof(float) * G * TB * out);
+    bytes += Workspace::up(sizeof(double) * Gtot);
+    bytes += Workspace::up(sizeof(double) * awq::reduce_scratch_doubles(G, out));
+    bytes += Workspace::up(sizeof(int) * 8);
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(bytes)) return s;
+    uint16_t *x16 = ws.take<uint16_t>(N * in);
+    float *s_tab = ws.take<float>(G * in);
+    float *inv_s_tab = ws.take<float>(G * in);
+    float4 *qparam = ws.take<float4>(G * out * nG);
+    float *part = ws.take<float>(G * TB * out);
+    double *loss_d = ws.take<double>(Gtot);
+    double *blocksum = ws.take<double>(awq::reduce_scratch_doubles(G, out));
+    // [0] best alpha, [1] best clip, [2] device error word, [3] max|X| bits, [4] X exponent
+    int *flags = ws.take<int>(8);
+    AWQ_CUDA(cudaMemsetAsync(flags, 0, sizeof(int) * 8, st));
+
+    AWQ_CUDA(awq::launch_x_to_f16(X, x_dtype == AWQ_BF16, N * in, reinterpret_cast<unsigned *>(flags + 3),
+                                  flags + 4, x16, st));
+    CUtensorMap xmap;
+    if (awq_status_t s = make_x_map(&xmap, x16, N, in)) return s;
+
+    awq::SearchArgs a{};
+    a.W = W;
+    a.w_bf16 = w_dtype == AWQ_BF16;
+    a.O = out;
+    a.I = in;
+    a.N = N;
+    a.gs = group_size;
+    a.s_tab = s_tab;
+    a.inv_s_tab = inv_s_tab;
+    a.qparam = qparam;
+    a.part = part;
+    a.err = flags + 2;
+
+    // Phase 1: the alpha grid (clip 1).
+    awq::GridParams ap{}, cp{};
+    for (int k = 0; k < n_alpha; ++k) {
+        ap.value[k] = alpha[k];
+        cp.value[k] = 1.0;
+    }
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, s_tab, inv_s_tab, st));
+    AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM, s_tab,
+                                      cp, n_alpha, qparam, st));
+    a.G = n_alpha;
+    a.clamp = quant == AWQ_ASYM;
+    kt_reset(1);
+    kt_begin(1, st);
+    AWQ_CUDA(awq::launch_search(a, xmap, sms, st));
+    kt_end(1, st);
+    AWQ_CUDA(awq::launch_reduce_loss(part, n_alpha, TB, out, N, flags + 4, loss_d, loss_row, blocksum,
+                                     st));
+    AWQ_CUDA(awq::launch_argmin(loss_d, n_alpha, flags + 0, st));
+
+    // Phase 2: the clip grid at alpha*.
+    if (n_clip > 0) {
+        awq::GridParams cp2{};
+        for (int k = 0; k < n_clip; ++k) cp2.value[k] = clip[k];
+        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, s_tab, inv_s_tab, st));
+        AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM,
+                                          s_tab, cp2, n_clip, qparam, st));
+        a.G = n_clip;
+        a.clamp = true;
+        kt_begin(1, st);
+        AWQ_CUDA(awq::launch_search(a, xmap, sms, st));
+        kt_end(1, st);
+        AWQ_CUDA(awq::launch_reduce_loss(part, n_clip, TB, out, N, flags + 4, loss_d + n_alpha,
+                                         loss_row ? loss_row + static_cast<int64_t>(n_alpha) * out
+                                                  : nullptr,
+                                         blocksum, st));
+        AWQ_CUDA(awq::launch_argmin(loss_d + n_alpha, n_clip, flags + 1, st));
+    }
+
+    int hflags[4];
+    AWQ_CUDA(cudaMemcpyAsync(loss, loss_d, sizeof(double) * Gtot, cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaMemcpyAsync(hflags, flags, sizeof(int) * 4, cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaStreamSynchronize(st));
+    if (hflags[2] != 0)
+        return fail(AWQ_ERR_TIMEOUT, "search kernel: a bounded wait gave up (device error %d)", hflags[2]);
+    *best_alpha = hflags[0];
+    *best_clip = n_clip > 0 ? hflags[1] : -1;
+    return AWQ_OK;
+}
+
+awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, const float *sX,
+                           double alpha, double clip, int group_size, int quant, uint32_t *qweight,
+                           uint16_t *scales, uint32_t *zeros, uint16_t *s16, float *scales_f32,
+                           void *stream) {
+    g_last_error.clear();
+    if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
+    if (!sX || !qweight || !scales || !s16) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (quant == AWQ_ASYM && !zeros) return fail(AWQ_ERR_ARG, "zeros required for AWQ_ASYM");
+    if (quant == AWQ_SYM && zeros) return fail(AWQ_ERR_ARG, "zeros must be NULL for AWQ_SYM");
+    if (!(alpha >= 0.0 && alpha <= 1.0)) return fail(AWQ_ERR_ARG, "alpha out of [0,1]");
+    if (!(clip > 0.0 && clip <= 1.0)) return fail(AWQ_ERR_ARG, "clip out of (0,1]");
+    if (!aligned16(sX) || !aligned16(qweight) || !aligned16(s16) ||
+        (scales_f32 && (reinterpret_cast<uintptr_t>(scales_f32) & 3u)) ||
+        (reinterpret_cast<uintptr_t>(scales) & 1u) || (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)))
+        return fail(AWQ_ERR_ALIGN, "misaligned pointer");
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(2 * Workspace::up(sizeof(float) * in))) return s;
+    float *s = ws.take<float>(in);
+    float *inv_s = ws.take<float>(in);
+    awq::GridParams ap{};
+    ap.value[0] = alpha;
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, s, inv_s, st));
+    const int64_t nG = in / group_size;
+    if (zeros) AWQ_CUDA(cudaMemsetAsync(zeros, 0, sizeof(uint32_t) * out * ((nG + 7) / 8), st));
+    kt_reset(2);
+    kt_begin(2, st);
+    AWQ_CUDA(awq::launch_pack(W, w_dtype == AWQ_BF16, out, in, group_size, quant == AWQ_ASYM, clip,
+                              s, qweight, scales, zeros, s16, scales_f32, st));
+    kt_end(2, st);
+    return AWQ_OK;
+}
+
+awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
+                              const uint32_t *qweight, const uint16_t *scales,
+                              const uint32_t *zeros, const uint16_t *s16, int group_size,
+                              uint16_t *y, void *stream) {
+    g_last_error.clear();
+    if (!x || !qweight || !scales || !s16 || !y) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (M < 1 || in < 1 || out < 1) return fail(AWQ_ERR_ARG, "bad shape");
+    if (group_size != 32 && group_size != 64 && group_size != 128)
+        return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
+    if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 64", (long long)in);
+    if (in > 13312) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld above 13312", (long long)in);
+    if (!aligned16(x) || !aligned16(qweight) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+        (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)) || !aligned16(s16) ||
+        (reinterpret_cast<uintptr_t>(y) & 1u))
+        return fail(AWQ_ERR_ALIGN, "misaligned pointer");
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kt_reset(3);
+    kt_begin(3, st);
+    AWQ_CUDA(awq::launch_w4a16(x, M, in, out, qweight, scales, zeros, s16, group_size, y, st));
+    kt_end(3, st);
+    return AWQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,80 @@
+// Internal launch interface between the C-ABI layer (awq_api.cu) and the
+// kernels.  Every launcher enqueues on `st` and returns the launch status.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace awq {
+
+constexpr int STATS_CHUNK = 128;   // tokens per fp64 partial sum of mean|X|
+constexpr int MAX_GRID = 64;       // grid points per search phase
+
+// Search tile shape: 128 output rows x 512 tokens per work unit, K slabs of 64.
+constexpr int TILE_O = 128;
+constexpr int TILE_N = 512;
+constexpr int SUB_N = 256;
+constexpr int SLAB_K = 64;
+
+struct GridParams {
+    double value[MAX_GRID];   // alpha per grid point (phase 1) or clip ratio (phase 2)
+};
+
+// ---- statistics
+cudaError_t launch_stats_partial(const void *X, bool x_bf16, int64_t N, int64_t I, double *part,
+                                 cudaStream_t st);
+cudaError_t launch_stats_final(const double *part, int64_t N, int64_t I, float clamp_min,
+                               float *sX, cudaStream_t st);
+// fp16 copy of X scaled by 2^-k (k written to *k_out on the device); *max_bits zeroed by the caller.
+cudaError_t launch_x_to_f16(const void *X, bool x_bf16, int64_t n, unsigned *max_bits, int *k_out,
+                            uint16_t *dst, cudaStream_t st);
+
+// ---- scale table: s[g][i], inv_s[g][i] for G grid points.
+// alpha_of_g: alpha values per grid point; if best_idx != nullptr every row uses
+// alpha_all[*best_idx] instead (the second, clip phase).
+cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
+                               const int *best_idx, float *s_tab, float *inv_s_tab,
+                               cudaStream_t st);
+
+// ---- per-(grid point, row, group) quantiser parameters {Delta, 1/Delta, qlo, qhi}
+cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
+                                bool asym, const float *s_tab, const GridParams &clip, int G,
+                                float4 *qparam, cudaStream_t st);
+
+// ---- fused search
+struct SearchArgs {
+    const void *W;
+    bool w_bf16;
+    int64_t O, I, N;
+    int gs;
+    int G;
+    bool clamp;                 // asymmetric or clipped: clamp codes to [qlo, qhi]
+    const float *s_tab, *inv_s_tab;
+    const float4 *qparam;
+    float *part;                // [G][TB][O]
+    int *err;
+};
+cudaError_t launch_search(const SearchArgs &a, const CUtensorMap &xmap, int num_sms,
+                          cudaStream_t st);
+
+// ---- loss reduction and selection
+// blocksum: scratch of reduce_scratch_doubles(G, O) doubles.
+int64_t reduce_scratch_doubles(int G, int64_t O);
+// Row sums are multiplied by 2^(2 * *x_exp) (the exact undo of X's fp16 scaling).
+cudaError_t launch_reduce_loss(const float *part, int G, int64_t TB, int64_t O, int64_t N,
+                               const int *x_exp, double *loss, float *loss_row, double *blocksum,
+                               cudaStream_t st);
+cudaError_t launch_argmin(const double *loss, int G, int *best, cudaStream_t st);
+
+// ---- packing
+cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs, bool asym,
+                        double clip, const float *s, uint32_t *qweight, uint16_t *scales,
+                        uint32_t *zeros, uint16_t *s16, float *scales_f32, cudaStream_t st);
+
+// ---- W4A16 apply
+cudaError_t launch_w4a16(const uint16_t *x, int64_t M, int64_t I, int64_t O,
+                         const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
+                         const uint16_t *s16, int gs, uint16_t *y, cudaStream_t st);
+
+}  // namespace awq

@@ -1,0 +1,265 @@
+// Scale vectors, group quantiser parameters and INT4 packing.
+//
+//   s[i]  = s_X[i]^alpha / max_j s_X[j]^alpha      (paper summary, Method:
+//           s = s_X^alpha; AWQ guide, section 三, step 2: scale / scale.max())
+//   Delta = max|W*s| / 7 over a (row, group) for the symmetric quantizer, or
+//           (max - min) / 15 with zero point z = clamp(rint(-min/Delta), 0, 15)
+//           for the asymmetric one (AWQ guide, section 三, step 4; paper
+//           summary, Method, first equation); clip ratios scale the bounds.
+//
+// Everything that decides an integer (Delta, z, codes) uses IEEE fp32
+// operations with explicit rounding intrinsics, so no FMA contraction or
+// approximate divide can change a code.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "awq_internal.h"
+
+namespace awq {
+
+// ------------------------------------------------------------ scale table
+__global__ void __launch_bounds__(256) scale_table_kernel(const float *__restrict__ sX, int64_t I,
+                                                          GridParams alpha,
+                                                          const int *__restrict__ best_idx,
+                                                          float *__restrict__ s_tab,
+                                                          float *__restrict__ inv_s_tab) {
+    __shared__ double red[256];
+    const int g = blockIdx.x;
+    const double a = best_idx ? alpha.value[*best_idx] : alpha.value[g];
+    double m = 0.0;
+    for (int64_t i = threadIdx.x; i < I; i += blockDim.x)
+        m = fmax(m, pow(static_cast<double>(sX[i]), a));
+    red[threadIdx.x] = m;
+    __syncthreads();
+    for (int off = 128; off > 0; off >>= 1) {
+        if (threadIdx.x < off) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + off]);
+        __syncthreads();
+    }
+    m = red[0];
+    for (int64_t i = threadIdx.x; i < I; i += blockDim.x) {
+        const double t = pow(static_cast<double>(sX[i]), a);
+        const float s = __double2float_rn(__ddiv_rn(t, m));
+        s_tab[g * I + i] = s;
+        inv_s_tab[g * I + i] = __frcp_rn(s);
+    }
+}
+
+cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
+                               const int *best_idx, float *s_tab, float *inv_s_tab,
+                               cudaStream_t st) {
+    scale_table_kernel<<<G, 256, 0, st>>>(sX, I, alpha, best_idx, s_tab, inv_s_tab);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------- group quantiser params
+__device__ __forceinline__ float clip_bound(float b, double r) {
+    return r == 1.0 ? b : __double2float_rn(__dmul_rn(static_cast<double>(b), r));
+}
+
+__device__ __forceinline__ float safe_rcp(float d) {
+    if (!(d > 0.0f)) return 0.0f;
+    const float r = __frcp_rn(d);
+    return isinf(r) ? 3.4028234663852886e38f : r;
+}
+
+// One warp per (row, group); each lane holds gs/32 elements of the group and
+// loops over the G grid points, so W is read once for all of them.
+template <bool WBF16, int EPL>
+__global__ void __launch_bounds__(256) group_params_kernel(
+    const void *__restrict__ W, int64_t O, int64_t I, int gs, bool asym,
+    const float *__restrict__ s_tab, GridParams clip, int G, float4 *__restrict__ qparam) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nG = I / gs;
+    const int64_t pair = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+    if (pair >= O * nG) return;
+    const int64_t o = pair / nG, j = pair % nG;
+    const int64_t col = j * gs + static_cast<int64_t>(lane) * EPL;
+    float w[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+        if constexpr (WBF16) {
+            const uint16_t b = static_cast<const uint16_t *>(W)[o * I + col + e];
+            w[e] = __uint_as_float(static_cast<uint32_t>(b) << 16);
+        } else {
+            w[e] = static_cast<const float *>(W)[o * I + col + e];
+        }
+    }
+    for (int g = 0; g < G; ++g) {
+        const float *s = s_tab + static_cast<int64_t>(g) * I + col;
+        float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+            const float wp = __fmul_rn(w[e], s[e]);
+            mx = fmaxf(mx, wp);
+            mn = fminf(mn, wp);
+            amax = fmaxf(amax, fabsf(wp));
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        }
+        if (lane == 0) {
+            const double r = clip.value[g];
+            float D, qlo, qhi;
+            if (!asym) {
+                D = __fdiv_rn(clip_bound(amax, r), 7.0f);
+                qlo = -8.0f;
+                qhi = 7.0f;
+            } else {
+                const float hi = clip_bound(mx, r), lo = clip_bound(mn, r);
+                D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+                float z = 0.0f;
+                if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+                qlo = -z;
+                qhi = 15.0f - z;
+                if (D == 0.0f) qhi = 0.0f;
+            }
+            qparam[(static_cast<int64_t>(g) * O + o) * nG + j] =
+                make_float4(D, safe_rcp(D), qlo, qhi);
+        }
+    }
+}
+
+cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
+                                bool asym, const float *s_tab, const GridParams &clip, int G,
+                                float4 *qparam, cudaStream_t st) {
+    const int64_t pairs = O * (I / gs);
+    const unsigned blocks = static_cast<unsigned>((pairs + 7) / 8);
+#define AWQ_GP(WB, E) \
+    group_params_kernel<WB, E><<<blocks, 256, 0, st>>>(W, O, I, gs, asym, s_tab, clip, G, qparam)
+    if (w_bf16) {
+        if (gs == 32) AWQ_GP(true, 1);
+        else if (gs == 64) AWQ_GP(true, 2);
+        else AWQ_GP(true, 4);
+    } else {
+        if (gs == 32) AWQ_GP(false, 1);
+        else if (gs == 64) AWQ_GP(false, 2);
+        else AWQ_GP(false, 4);
+    }
+#undef AWQ_GP
+    return cudaGetLastError();
+}
+
+// -------------------------------------------------------------------- pack
+// One thread per packed word (8 consecutive columns of a row).  The gs/8
+// threads of a group are consecutive lanes of one warp and reduce with xor
+// shuffles; the first of them writes the group's scale and zero point.
+template <bool WBF16>
+__global__ void __launch_bounds__(256) pack_kernel(const void *__restrict__ W, int64_t O, int64_t I,
+                                                   int gs, bool asym, double clip,
+                                                   const float *__restrict__ s,
+                                                   uint32_t *__restrict__ qweight,
+                                                   uint16_t *__restrict__ scales,
+                                                   uint32_t *__restrict__ zeros,
+                                                   uint16_t *__restrict__ s16,
+                                                   float *__restrict__ scales_f32) {
+    const int64_t wpr = I / 8;
+    const int64_t total = O * wpr;
+    const int seg = gs / 8;
+    const int64_t nG = I / gs;
+    const int64_t nzw = (nG + 7) / 8;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t iters = (total + step - 1) / step;
+    for (int64_t it = 0; it < iters; ++it) {
+        const int64_t idx = it * step + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+        const bool active = idx < total;
+        const int64_t o = active ? idx / wpr : 0;
+        const int64_t wcol = active ? idx % wpr : 0;
+        const int64_t c0 = wcol * 8;
+        float w[8], sv[8], wp[8];
+        if (active) {
+            if constexpr (WBF16) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(W) +
+                                                                o * I + c0);
+                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    w[2 * k] = __uint_as_float(u[k] << 16);
+                    w[2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
+                }
+            } else {
+                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(W) +
+                                                                  o * I + c0);
+                const float4 a = p[0], b = p[1];
+                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+                w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+            }
+            const float4 sa = *reinterpret_cast<const float4 *>(s + c0);
+            const float4 sb = *reinterpret_cast<const float4 *>(s + c0 + 4);
+            sv[0] = sa.x; sv[1] = sa.y; sv[2] = sa.z; sv[3] = sa.w;
+            sv[4] = sb.x; sv[5] = sb.y; sv[6] = sb.z; sv[7] = sb.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) { w[k] = 0.0f; sv[k] = 1.0f; }
+        }
+        float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            wp[k] = __fmul_rn(w[k], sv[k]);
+            mx = fmaxf(mx, wp[k]);
+            mn = fminf(mn, wp[k]);
+            amax = fmaxf(amax, fabsf(wp[k]));
+        }
+        for (int off = 1; off < seg; off <<= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        }
+        float D, z = 0.0f;
+        uint32_t word = 0;
+        if (!asym) {
+            const float a = clip == 1.0 ? amax : __double2float_rn(__dmul_rn((double)amax, clip));
+            D = __fdiv_rn(a, 7.0f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float q = 0.0f;
+                if (D != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(wp[k], D)), -8.0f), 7.0f);
+                word |= (static_cast<uint32_t>(static_cast<int>(q) + 8) & 0xFu) << (4 * k);
+            }
+        } else {
+            const float hi = clip == 1.0 ? mx : __double2float_rn(__dmul_rn((double)mx, clip));
+            const float lo = clip == 1.0 ? mn : __double2float_rn(__dmul_rn((double)mn, clip));
+            D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+            if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                float q = 0.0f;
+                if (D != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(wp[k], D)) + z, 0.0f), 15.0f);
+                word |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xFu) << (4 * k);
+            }
+        }
+        if (!active) continue;
+        qweight[idx] = word;
+        if ((wcol % seg) == 0) {
+            const int64_t j = c0 / gs;
+            scales[o * nG + j] = __half_as_ushort(__float2half_rn(D));
+            if (scales_f32) scales_f32[o * nG + j] = D;
+            if (zeros)
+                atomicOr(&zeros[o * nzw + j / 8],
+                         (static_cast<uint32_t>(z) & 0xFu) << (4 * static_cast<int>(j % 8)));
+        }
+        if (o == 0) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) s16[c0 + k] = __half_as_ushort(__float2half_rn(sv[k]));
+        }
+    }
+}
+
+cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs, bool asym,
+                        double clip, const float *s, uint32_t *qweight, uint16_t *scales,
+                        uint32_t *zeros, uint16_t *s16, float *scales_f32, cudaStream_t st) {
+    const int64_t total = O * (I / 8);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (w_bf16)
+        pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            W, O, I, gs, asym, clip, s, qweight, scales, zeros, s16, scales_f32);
+    else
+        pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            W, O, I, gs, asym, clip, s, qweight, scales, zeros, s16, scales_f32);
+    return cudaGetLastError();
+}
+
+}  // namespace awq
