@@ -39,11 +39,11 @@ class AwqError(RuntimeError):
         self.status_name = status_name
 
 
-def _load_library() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+def _load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python weight_only_quantization_awq_b200/build.py`")
-    lib = ctypes.CDLL(LIB_PATH)
+            f"{path} is not built; run `python weight_only_quantization_awq_b200/build.py`")
+    lib = ctypes.CDLL(path)
     P, I, L, F, D = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
                      ctypes.c_double)
     lib.awq_version.restype = I

@@ -11,7 +11,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/awq_b200.h"
+#include "awq_b200.h"
 #include "awq_internal.h"
 
 namespace {
@@ -109,21 +109,48 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// Tensor map of the fp16 copy of X [N, I]: boxes of 64 channels x 256 tokens, 128-byte
-// swizzle (the K-major layout the MMA descriptors describe), zero fill out of
-// bounds so ragged token tails contribute nothing.
-awq_status_t make_x_map(CUtensorMap *map, const void *X, int64_t N, int64_t I) {
+// A 2-D tiled tensor map over a row-major [dim1, dim0] array.
+awq_status_t make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, size_t elem, const void *ptr,
+                         uint64_t dim0, uint64_t dim1, uint32_t box0, uint32_t box1,
+                         CUtensorMapSwizzle swz) {
     auto enc = get_encode();
     if (!enc) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(I), static_cast<cuuint64_t>(N)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(I) * 2};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(awq::SLAB_K), static_cast<cuuint32_t>(awq::SUB_N)};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(dim0), static_cast<cuuint64_t>(dim1)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(dim0 * elem)};
+    cuuint32_t box[2] = {box0, box1};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(X), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = enc(map, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return AWQ_OK;
+}
+
+// The search kernel's four tensor maps (out-of-bounds boxes read as zero, so
+// ragged rows and token tails contribute nothing):
+//   x  : fp16 copy of X [N, I], boxes of 64 channels x 256 tokens, 128B swizzle;
+//   w  : W [O, I], 128 rows x 128 bytes per box, 128B swizzle;
+//   sn : scale table [2G, I] fp32, boxes of 64 channels x (s row, -1/s row);
+//   qp : group parameters [G*O, 4*I/gs] fp32, boxes of 128 rows x the groups
+//        one 64-column slab touches.
+awq_status_t make_search_maps(awq::SearchMaps *m, const uint16_t *x16, int64_t N, const void *W,
+                              bool w_bf16, int64_t O, int64_t I, const float *sn,
+                              const float4 *qparam, int G, int gs) {
+    if (awq_status_t s = make_map_2d(&m->x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, I, N,
+                                     awq::SLAB_K, awq::SUB_N, CU_TENSOR_MAP_SWIZZLE_128B))
+        return s;
+    if (awq_status_t s = w_bf16 ? make_map_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, I, O,
+                                              64, awq::TILE_O, CU_TENSOR_MAP_SWIZZLE_128B)
+                                : make_map_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, I, O,
+                                              32, awq::TILE_O, CU_TENSOR_MAP_SWIZZLE_128B))
+        return s;
+    if (awq_status_t s = make_map_2d(&m->sn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sn, I, 2 * G,
+                                     awq::SLAB_K, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return s;
+    const int gps = gs == 32 ? 2 : 1;
+    return make_map_2d(&m->qp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, qparam, 4 * (I / gs),
+                       static_cast<uint64_t>(G) * O, 4 * gps, awq::TILE_O,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 bool valid_dtype(int d) { return d == AWQ_F32 || d == AWQ_BF16; }
@@ -273,7 +300,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     const int Gtot = n_alpha + n_clip;
     size_t bytes = 0;
     bytes += Workspace::up(sizeof(uint16_t) * N * in);
-    bytes += 2 * Workspace::up(sizeof(float) * G * in);
+    bytes += Workspace::up(sizeof(float) * 2 * G * in);
     bytes += Workspace::up(sizeof(float4) * G * out * nG);
     bytes += Workspace::up(sizeof(float) * G * TB * out);
     bytes += Workspace::up(sizeof(double) * Gtot);
@@ -282,8 +309,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     Workspace ws(st);
     if (awq_status_t s = ws.reserve(bytes)) return s;
     uint16_t *x16 = ws.take<uint16_t>(N * in);
-    float *s_tab = ws.take<float>(G * in);
-    float *inv_s_tab = ws.take<float>(G * in);
+    float *sn = ws.take<float>(2 * G * in);
     float4 *qparam = ws.take<float4>(G * out * nG);
     float *part = ws.take<float>(G * TB * out);
     double *loss_d = ws.take<double>(Gtot);
@@ -294,21 +320,15 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
 
     AWQ_CUDA(awq::launch_x_to_f16(X, x_dtype == AWQ_BF16, N * in, reinterpret_cast<unsigned *>(flags + 3),
                                   flags + 4, x16, st));
-    CUtensorMap xmap;
-    if (awq_status_t s = make_x_map(&xmap, x16, N, in)) return s;
-
     awq::SearchArgs a{};
-    a.W = W;
     a.w_bf16 = w_dtype == AWQ_BF16;
     a.O = out;
     a.I = in;
     a.N = N;
     a.gs = group_size;
-    a.s_tab = s_tab;
-    a.inv_s_tab = inv_s_tab;
-    a.qparam = qparam;
     a.part = part;
     a.err = flags + 2;
+    awq::SearchMaps maps;
 
     // Phase 1: the alpha grid (clip 1).
     awq::GridParams ap{}, cp{};
@@ -316,14 +336,17 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
         ap.value[k] = alpha[k];
         cp.value[k] = 1.0;
     }
-    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, s_tab, inv_s_tab, st));
-    AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM, s_tab,
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, sn, st));
+    AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM, sn,
                                       cp, n_alpha, qparam, st));
     a.G = n_alpha;
     a.clamp = quant == AWQ_ASYM;
+    if (awq_status_t s = make_search_maps(&maps, x16, N, W, a.w_bf16, out, in, sn, qparam, n_alpha,
+                                          group_size))
+        return s;
     kt_reset(1);
     kt_begin(1, st);
-    AWQ_CUDA(awq::launch_search(a, xmap, sms, st));
+    AWQ_CUDA(awq::launch_search(a, maps, sms, st));
     kt_end(1, st);
     AWQ_CUDA(awq::launch_reduce_loss(part, n_alpha, TB, out, N, flags + 4, loss_d, loss_row, blocksum,
                                      st));
@@ -333,13 +356,16 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     if (n_clip > 0) {
         awq::GridParams cp2{};
         for (int k = 0; k < n_clip; ++k) cp2.value[k] = clip[k];
-        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, s_tab, inv_s_tab, st));
+        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, sn, st));
         AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM,
-                                          s_tab, cp2, n_clip, qparam, st));
+                                          sn, cp2, n_clip, qparam, st));
         a.G = n_clip;
         a.clamp = true;
+        if (awq_status_t s = make_search_maps(&maps, x16, N, W, a.w_bf16, out, in, sn, qparam,
+                                              n_clip, group_size))
+            return s;
         kt_begin(1, st);
-        AWQ_CUDA(awq::launch_search(a, xmap, sms, st));
+        AWQ_CUDA(awq::launch_search(a, maps, sms, st));
         kt_end(1, st);
         AWQ_CUDA(awq::launch_reduce_loss(part, n_clip, TB, out, N, flags + 4, loss_d + n_alpha,
                                          loss_row ? loss_row + static_cast<int64_t>(n_alpha) * out
@@ -378,18 +404,17 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, 
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Workspace ws(st);
-    if (awq_status_t s = ws.reserve(2 * Workspace::up(sizeof(float) * in))) return s;
-    float *s = ws.take<float>(in);
-    float *inv_s = ws.take<float>(in);
+    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(float) * 2 * in))) return s;
+    float *sn = ws.take<float>(2 * in);   // row 0: s, row 1: -1/s
     awq::GridParams ap{};
     ap.value[0] = alpha;
-    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, s, inv_s, st));
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, sn, st));
     const int64_t nG = in / group_size;
     if (zeros) AWQ_CUDA(cudaMemsetAsync(zeros, 0, sizeof(uint32_t) * out * ((nG + 7) / 8), st));
     kt_reset(2);
     kt_begin(2, st);
     AWQ_CUDA(awq::launch_pack(W, w_dtype == AWQ_BF16, out, in, group_size, quant == AWQ_ASYM, clip,
-                              s, qweight, scales, zeros, s16, scales_f32, st));
+                              sn, qweight, scales, zeros, s16, scales_f32, st));
     kt_end(2, st);
     return AWQ_OK;
 }

@@ -30,32 +30,36 @@ cudaError_t launch_stats_final(const double *part, int64_t N, int64_t I, float c
 cudaError_t launch_x_to_f16(const void *X, bool x_bf16, int64_t n, unsigned *max_bits, int *k_out,
                             uint16_t *dst, cudaStream_t st);
 
-// ---- scale table: s[g][i], inv_s[g][i] for G grid points.
-// alpha_of_g: alpha values per grid point; if best_idx != nullptr every row uses
-// alpha_all[*best_idx] instead (the second, clip phase).
+// ---- scale table sn[G][2][I]: row 2g holds s_g, row 2g+1 holds -1/s_g.
+// alpha.value[g] is grid point g's alpha; if best_idx != nullptr every row uses
+// alpha.value[*best_idx] instead (the second, clip phase).
 cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
-                               const int *best_idx, float *s_tab, float *inv_s_tab,
-                               cudaStream_t st);
+                               const int *best_idx, float *sn, cudaStream_t st);
 
-// ---- per-(grid point, row, group) quantiser parameters {Delta, 1/Delta, qlo, qhi}
+// ---- per-(grid point, row, group) quantiser parameters {Delta, 1/Delta, -qhi, -qlo}
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
-                                bool asym, const float *s_tab, const GridParams &clip, int G,
+                                bool asym, const float *sn, const GridParams &clip, int G,
                                 float4 *qparam, cudaStream_t st);
 
 // ---- fused search
+// Tensor maps of the kernel's four inputs:
+//   x  : fp16 copy of X [N, I], box 64 x 256, 128B swizzle
+//   w  : W [O, I] (bf16: box 64 x 128; fp32: box 32 x 128), 128B swizzle
+//   sn : scale table [2G, I] fp32, box 64 x 2
+//   qp : group parameters [G*O, 4*I/gs] fp32, box (4 * groups per slab) x 128
+struct SearchMaps {
+    CUtensorMap x, w, sn, qp;
+};
 struct SearchArgs {
-    const void *W;
-    bool w_bf16;
     int64_t O, I, N;
     int gs;
     int G;
+    bool w_bf16;
     bool clamp;                 // asymmetric or clipped: clamp codes to [qlo, qhi]
-    const float *s_tab, *inv_s_tab;
-    const float4 *qparam;
     float *part;                // [G][TB][O]
     int *err;
 };
-cudaError_t launch_search(const SearchArgs &a, const CUtensorMap &xmap, int num_sms,
+cudaError_t launch_search(const SearchArgs &a, const SearchMaps &maps, int num_sms,
                           cudaStream_t st);
 
 // ---- loss reduction and selection

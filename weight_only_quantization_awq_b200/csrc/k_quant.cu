@@ -21,8 +21,7 @@ namespace awq {
 __global__ void __launch_bounds__(256) scale_table_kernel(const float *__restrict__ sX, int64_t I,
                                                           GridParams alpha,
                                                           const int *__restrict__ best_idx,
-                                                          float *__restrict__ s_tab,
-                                                          float *__restrict__ inv_s_tab) {
+                                                          float *__restrict__ sn) {
     __shared__ double red[256];
     const int g = blockIdx.x;
     const double a = best_idx ? alpha.value[*best_idx] : alpha.value[g];
@@ -39,15 +38,14 @@ __global__ void __launch_bounds__(256) scale_table_kernel(const float *__restric
     for (int64_t i = threadIdx.x; i < I; i += blockDim.x) {
         const double t = pow(static_cast<double>(sX[i]), a);
         const float s = __double2float_rn(__ddiv_rn(t, m));
-        s_tab[g * I + i] = s;
-        inv_s_tab[g * I + i] = __frcp_rn(s);
+        sn[(2 * g) * I + i] = s;
+        sn[(2 * g + 1) * I + i] = -__frcp_rn(s);
     }
 }
 
 cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
-                               const int *best_idx, float *s_tab, float *inv_s_tab,
-                               cudaStream_t st) {
-    scale_table_kernel<<<G, 256, 0, st>>>(sX, I, alpha, best_idx, s_tab, inv_s_tab);
+                               const int *best_idx, float *sn, cudaStream_t st) {
+    scale_table_kernel<<<G, 256, 0, st>>>(sX, I, alpha, best_idx, sn);
     return cudaGetLastError();
 }
 
@@ -67,7 +65,7 @@ __device__ __forceinline__ float safe_rcp(float d) {
 template <bool WBF16, int EPL>
 __global__ void __launch_bounds__(256) group_params_kernel(
     const void *__restrict__ W, int64_t O, int64_t I, int gs, bool asym,
-    const float *__restrict__ s_tab, GridParams clip, int G, float4 *__restrict__ qparam) {
+    const float *__restrict__ sn, GridParams clip, int G, float4 *__restrict__ qparam) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nG = I / gs;
     const int64_t pair = static_cast<int64_t>(blockIdx.x) * 8 + warp;
@@ -85,7 +83,7 @@ __global__ void __launch_bounds__(256) group_params_kernel(
         }
     }
     for (int g = 0; g < G; ++g) {
-        const float *s = s_tab + static_cast<int64_t>(g) * I + col;
+        const float *s = sn + static_cast<int64_t>(2 * g) * I + col;
         float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -116,19 +114,20 @@ __global__ void __launch_bounds__(256) group_params_kernel(
                 qhi = 15.0f - z;
                 if (D == 0.0f) qhi = 0.0f;
             }
+            // {Delta, 1/Delta, -qhi, -qlo}: the search kernel works with -q.
             qparam[(static_cast<int64_t>(g) * O + o) * nG + j] =
-                make_float4(D, safe_rcp(D), qlo, qhi);
+                make_float4(D, safe_rcp(D), -qhi, -qlo);
         }
     }
 }
 
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
-                                bool asym, const float *s_tab, const GridParams &clip, int G,
+                                bool asym, const float *sn, const GridParams &clip, int G,
                                 float4 *qparam, cudaStream_t st) {
     const int64_t pairs = O * (I / gs);
     const unsigned blocks = static_cast<unsigned>((pairs + 7) / 8);
 #define AWQ_GP(WB, E) \
-    group_params_kernel<WB, E><<<blocks, 256, 0, st>>>(W, O, I, gs, asym, s_tab, clip, G, qparam)
+    group_params_kernel<WB, E><<<blocks, 256, 0, st>>>(W, O, I, gs, asym, sn, clip, G, qparam)
     if (w_bf16) {
         if (gs == 32) AWQ_GP(true, 1);
         else if (gs == 64) AWQ_GP(true, 2);

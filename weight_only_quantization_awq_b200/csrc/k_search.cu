@@ -4,24 +4,25 @@
 // [512*tb, 512*tb + 512), it accumulates
 //     E[o, n] = sum_i dW_g[o, i] * X[n, i],   dW_g = Q(W * s_g) / s_g - W
 // on the 5th-generation tensor cores (fp16 operands, fp32 accumulation) and
-// reduces sum_n E[o, n]^2 per row.
-// This is the objective L(s) = ||Q(W*s)(s^-1*X) - W X|| of the AWQ paper
-// summary (Method), with the 1/s moved from X's columns onto the weight
-// columns (exact in real arithmetic), evaluated for every s = s_X^alpha on the
-// grid.  Neither dW nor E ever reaches global memory.
+// reduces sum_n E[o, n]^2 per row.  This is the objective
+// L(s) = ||Q(W*s)(s^-1*X) - W X|| of the AWQ paper summary (Method), with the
+// 1/s moved from X's columns onto the weight columns (exact in real
+// arithmetic), evaluated for every s = s_X^alpha on the grid.  Neither dW nor E
+// ever reaches global memory.
 //
 // Warp roles (448 threads, one CTA per SM, persistent over work units):
-//   warps 0-7   dW producers: read W (bf16/fp32) and the per-group quantiser
-//               parameters, form dW for a 128 x 64 slab in registers, write it
-//               as fp16 into shared memory in the 128-byte-swizzled K-major
-//               layout the MMA reads, then signal a_full.
+//   warps 0-7   dW producers: read one slab's inputs (W tile, s and -1/s, group
+//               parameters) from shared memory, form dW for 128 rows x 64
+//               columns, write it as fp16 into shared memory in the
+//               128-byte-swizzled K-major layout the MMA reads, signal a_full.
 //   warps 8-11  epilogue: tcgen05.ld of the 128 x 512 fp32 accumulator (lane =
 //               output row), square-and-sum per row, one fp32 partial per
 //               (grid point, token block, row).
-//   warp 12     TMA: X tiles of 256 tokens x 64 channels (fp16 copy of X scaled
-//               by a power of two, 128B swizzle) into a 5-stage ring.
-//   warp 13     MMA: allocates 512 TMEM columns, one elected thread issues
-//               tcgen05.mma M=128 N=256 K=16 (two N=256 halves per slab), and
+//   warp 12     TMA: lane 0 streams X tiles (256 tokens x 64 channels, fp16
+//               copy of X scaled by a power of two) into the X ring; lane 1
+//               streams each slab's producer inputs into the input ring.
+//   warp 13     MMA: allocates 512 TMEM columns; one thread issues
+//               tcgen05.mma M=128 N=256 K=16 (two N=256 halves per slab) and
 //               tcgen05.commit releases ring stages and the accumulator.
 // Work units are (g fastest, then output tile, then token block) and are dealt
 // round-robin to the CTAs, so the CTAs running at one time share a few W tiles
@@ -39,15 +40,29 @@ constexpr int NUM_PRODUCER_WARPS = 8;
 constexpr int WARP_TMA = 12;
 constexpr int WARP_MMA = 13;
 constexpr int NUM_THREADS = 14 * 32;
-constexpr int XS = 5;                                  // X ring stages
-constexpr int AS = 3;                                  // dW ring stages
-constexpr int X_STAGE_BYTES = SUB_N * SLAB_K * 2;      // 32 KB
-constexpr int A_STAGE_BYTES = TILE_O * SLAB_K * 2;     // 16 KB
-constexpr int NUM_BARS = 2 * XS + 2 * AS + 3;
-constexpr int SMEM_BYTES = 1024 + XS * X_STAGE_BYTES + AS * A_STAGE_BYTES + NUM_BARS * 8 + 16;
+constexpr int X_STAGE_BYTES = SUB_N * SLAB_K * 2;      // 32 KB of fp16 X
+constexpr int A_STAGE_BYTES = TILE_O * SLAB_K * 2;     // 16 KB of fp16 dW
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_f16_f32(TILE_O, SUB_N, false);
 constexpr float MAGIC = 12582912.0f;                   // 1.5 * 2^23: x + MAGIC - MAGIC = rint(x)
+
+// Shared-memory plan, per weight type.  Input stage = W tile, then s / -1/s of
+// the slab (2 x 64 fp32), then the 128 rows' group parameters (1 or 2 float4).
+template <bool WBF16>
+struct Plan {
+    static constexpr int XS = WBF16 ? 4 : 3;            // X ring stages
+    static constexpr int AS = 2;                        // dW ring stages
+    static constexpr int IS = WBF16 ? 3 : 2;            // input ring stages
+    static constexpr int W_BYTES = WBF16 ? 16384 : 32768;
+    static constexpr int SN_OFF = W_BYTES;
+    static constexpr int QP_OFF = SN_OFF + 512;
+    static constexpr int IN_STAGE = ((QP_OFF + 4096) + 1023) / 1024 * 1024;
+    static constexpr int NUM_BARS = 2 * XS + 2 * AS + 2 * IS + 3;
+    static constexpr int SMEM_BYTES =
+        1024 + XS * X_STAGE_BYTES + AS * A_STAGE_BYTES + IS * IN_STAGE + NUM_BARS * 8 + 16;
+};
+static_assert(Plan<true>::SMEM_BYTES <= 232448, "shared memory plan (bf16 W) too large");
+static_assert(Plan<false>::SMEM_BYTES <= 232448, "shared memory plan (fp32 W) too large");
 
 struct Unit {
     int g;
@@ -71,120 +86,161 @@ __device__ __forceinline__ Unit decode(int64_t u, const SearchArgs &a, int64_t O
 // W' * RN(1/Delta) and RN(W'/Delta) differ by at most 32 * 2^-23 = 2^-18.
 constexpr float TIE_BAND = 0.5f - 1.0f / 65536.0f;
 
-// dW for 8 adjacent columns of one row (one group), packed as 4 x fp16x2.
-// Codes follow the quantizer's definition q = rint(RN(W'/Delta)) exactly: the
-// fast path rounds W' * (1/Delta), and any element whose product lies within
-// 2^-16 of a half-integer (exact ties included) is redone with the correctly
-// rounded division, so the result never depends on the reciprocal.
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// dW for 8 adjacent columns of one row (one group), packed as 4 x fp16x2, on
+// packed f32x2 arithmetic.  With t = RN(W' * (1/Delta) + MAGIC):
+//   nq = MAGIC - t = -q exactly,   frac = W' * (1/Delta) - q,
+//   d  = W' - q*Delta,             dW = d * (-1/s) = (q*Delta - W') / s.
+// Codes follow the quantizer's definition q = rint(RN(W'/Delta)): any element
+// whose reciprocal product lies within 2^-16 of a half-integer (exact ties
+// included) is redone with the correctly rounded division.
+// prm = {Delta, 1/Delta, -qhi, -qlo}; ns = -1/s.
 template <bool CLAMP>
-__device__ __forceinline__ uint4 dw_chunk8(const float (&w)[8], const float (&s)[8],
-                                           const float (&is)[8], const float4 &prm) {
-    float wp[8], q[8];
-    bool near_tie = false;
+__device__ __forceinline__ uint4 dw_chunk8(const float (&w)[8], const float4 &s0, const float4 &s1,
+                                           const float4 &n0, const float4 &n1, const float4 &prm) {
+    const float2 invD = f2(prm.y, prm.y), D = f2(prm.x, prm.x);
+    const float2 M2 = f2(MAGIC, MAGIC), NEG1 = f2(-1.0f, -1.0f);
+    const float2 sv[4] = {f2(s0.x, s0.y), f2(s0.z, s0.w), f2(s1.x, s1.y), f2(s1.z, s1.w)};
+    const float2 nv[4] = {f2(n0.x, n0.y), f2(n0.z, n0.w), f2(n1.x, n1.y), f2(n1.z, n1.w)};
+    float2 wp[4], nq[4];
+    float worst = 0.0f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        wp[e] = __fmul_rn(w[e], s[e]);                                 // W * s
-        q[e] = __fsub_rn(__fmaf_rn(wp[e], prm.y, MAGIC), MAGIC);        // rint(W*s * (1/Delta))
-        near_tie |= fabsf(__fmaf_rn(wp[e], prm.y, -q[e])) > TIE_BAND;
+    for (int e = 0; e < 4; ++e) {
+        wp[e] = __fmul2_rn(f2(w[2 * e], w[2 * e + 1]), sv[e]);
+        const float2 t = __ffma2_rn(wp[e], invD, M2);
+        nq[e] = __ffma2_rn(t, NEG1, M2);
+        const float2 fr = __ffma2_rn(wp[e], invD, nq[e]);
+        worst = fmaxf(worst, fmaxf(fabsf(fr.x), fabsf(fr.y)));
     }
-    if (near_tie) {
+    if (worst > TIE_BAND) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (prm.x != 0.0f) q[e] = rintf(__fdiv_rn(wp[e], prm.x));
+        for (int e = 0; e < 4; ++e) {
+            if (prm.x != 0.0f) {
+                nq[e].x = -rintf(__fdiv_rn(wp[e].x, prm.x));
+                nq[e].y = -rintf(__fdiv_rn(wp[e].y, prm.x));
+            }
+        }
     }
-    float r[8];
+    uint32_t out[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        float qe = q[e];
-        if (CLAMP) qe = fminf(fmaxf(qe, prm.z), prm.w);                // code range
-        r[e] = __fmul_rn(__fmaf_rn(qe, prm.x, -wp[e]), is[e]);         // (q*Delta - W*s) / s
+    for (int e = 0; e < 4; ++e) {
+        float2 n = nq[e];
+        if (CLAMP) {
+            n.x = fminf(fmaxf(n.x, prm.z), prm.w);
+            n.y = fminf(fmaxf(n.y, prm.z), prm.w);
+        }
+        const float2 d = __ffma2_rn(n, D, wp[e]);        // W' - q*Delta
+        const float2 r = __fmul2_rn(d, nv[e]);           // (q*Delta - W') / s
+        out[e] = f16x2_satfinite(r.x, r.y);
     }
-    uint4 pk;
-    pk.x = f16x2_satfinite(r[0], r[1]);
-    pk.y = f16x2_satfinite(r[2], r[3]);
-    pk.z = f16x2_satfinite(r[4], r[5]);
-    pk.w = f16x2_satfinite(r[6], r[7]);
-    return pk;
+    return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 template <bool WBF16, bool CLAMP>
-__device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t OT, int64_t U,
-                                              uint8_t *a_ring, uint64_t *a_full, uint64_t *a_empty,
+__device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
+                                              const uint8_t *in_ring, uint64_t *in_full,
+                                              uint64_t *in_empty, uint8_t *a_ring,
+                                              uint64_t *a_full, uint64_t *a_empty,
                                               volatile int *abort_flag) {
+    using P = Plan<WBF16>;
     const int t = threadIdx.x;          // 0..255
     const int r = t >> 1, hc = t & 1;   // row in tile, half of the 64-wide slab
+    const int gps = a.gs == 32 ? 2 : 1; // group-parameter entries per row in a stage
+    const int jq = a.gs == 32 ? hc : 0; // this thread's entry
     const int64_t nK = a.I / SLAB_K;
-    const int64_t nG = a.I / a.gs;
     uint32_t it = 0;
     for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
-        const Unit un = decode(u, a, OT);
-        const int64_t row = un.ot * TILE_O + r;
-        const bool valid = row < a.O;
-        const float *srow = a.s_tab + static_cast<int64_t>(un.g) * a.I;
-        const float *isrow = a.inv_s_tab + static_cast<int64_t>(un.g) * a.I;
-        const float4 *qp = a.qparam + (static_cast<int64_t>(un.g) * a.O + (valid ? row : 0)) * nG;
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
-            const int64_t col0 = kb * SLAB_K + hc * 32;
-            uint32_t wraw[WBF16 ? 16 : 32];
-            if (valid) {
-                if constexpr (WBF16) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        static_cast<const uint16_t *>(a.W) + row * a.I + col0);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint4 v = __ldg(src + k);
-                        wraw[4 * k] = v.x; wraw[4 * k + 1] = v.y;
-                        wraw[4 * k + 2] = v.z; wraw[4 * k + 3] = v.w;
-                    }
-                } else {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        static_cast<const float *>(a.W) + row * a.I + col0);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint4 v = __ldg(src + k);
-                        wraw[4 * k] = v.x; wraw[4 * k + 1] = v.y;
-                        wraw[4 * k + 2] = v.z; wraw[4 * k + 3] = v.w;
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < (WBF16 ? 16 : 32); ++k) wraw[k] = 0u;
-            }
-            const float4 prm = valid ? __ldg(qp + col0 / a.gs) : make_float4(0.f, 0.f, 0.f, 0.f);
-
-            const uint32_t stage = it % AS, phase = (it / AS) & 1u;
-            if (!mbar_wait(&a_empty[stage], phase ^ 1u, abort_flag)) return;
-            uint8_t *dst = a_ring + stage * A_STAGE_BYTES;
+            const uint32_t is = it % P::IS, as = it % P::AS;
+            if (!mbar_wait(&in_full[is], (it / P::IS) & 1u, abort_flag)) return;
+            if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag)) return;
+            const uint8_t *in = in_ring + is * P::IN_STAGE;
+            uint8_t *dst = a_ring + as * A_STAGE_BYTES;
+            const float4 prm = reinterpret_cast<const float4 *>(in + P::QP_OFF)[r * gps + jq];
+            const float *s_sm = reinterpret_cast<const float *>(in + P::SN_OFF) + hc * 32;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const float4 s0 = __ldg(reinterpret_cast<const float4 *>(srow + col0 + 8 * c));
-                const float4 s1 = __ldg(reinterpret_cast<const float4 *>(srow + col0 + 8 * c + 4));
-                const float4 i0 = __ldg(reinterpret_cast<const float4 *>(isrow + col0 + 8 * c));
-                const float4 i1 = __ldg(reinterpret_cast<const float4 *>(isrow + col0 + 8 * c + 4));
-                const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-                const float iv[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-                float wv[8];
+                float w[8];
                 if constexpr (WBF16) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(in + sw128_offset(r, hc * 4 + c));
+                    const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t u2 = wraw[4 * c + k];
-                        wv[2 * k] = __uint_as_float(u2 << 16);
-                        wv[2 * k + 1] = __uint_as_float(u2 & 0xFFFF0000u);
+                        w[2 * k] = __uint_as_float(u4[k] << 16);
+                        w[2 * k + 1] = __uint_as_float(u4[k] & 0xFFFF0000u);
                     }
                 } else {
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) wv[k] = __uint_as_float(wraw[8 * c + k]);
+                    const uint8_t *sub = in + hc * 16384;   // columns hc*32 .. hc*32+31
+                    const float4 v0 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, 2 * c));
+                    const float4 v1 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, 2 * c + 1));
+                    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
                 }
+                const float4 s0 = *reinterpret_cast<const float4 *>(s_sm + 8 * c);
+                const float4 s1 = *reinterpret_cast<const float4 *>(s_sm + 8 * c + 4);
+                const float4 n0 = *reinterpret_cast<const float4 *>(s_sm + 64 + 8 * c);
+                const float4 n1 = *reinterpret_cast<const float4 *>(s_sm + 64 + 8 * c + 4);
                 *reinterpret_cast<uint4 *>(dst + sw128_offset(r, hc * 4 + c)) =
-                    dw_chunk8<CLAMP>(wv, sv, iv, prm);
+                    dw_chunk8<CLAMP>(w, s0, s1, n0, n1, prm);
             }
+            mbar_arrive(&in_empty[is]);
             fence_proxy_async_smem();
-            mbar_arrive(&a_full[stage]);
+            mbar_arrive(&a_full[as]);
         }
     }
 }
 
-__device__ __forceinline__ void tma_role(const SearchArgs &a, const CUtensorMap *xmap, int64_t OT,
+// Lane 1 of the TMA warp: the producers' inputs, one stage per (unit, slab).
+template <bool WBF16>
+__device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMaps &m, int64_t OT,
+                                             int64_t U, uint8_t *in_ring, uint64_t *in_full,
+                                             uint64_t *in_empty, volatile int *abort_flag) {
+    using P = Plan<WBF16>;
+    const int64_t nK = a.I / SLAB_K;
+    const int gps = a.gs == 32 ? 2 : 1;
+    const uint32_t bytes = P::W_BYTES + 512 + 2048 * gps;
+    uint32_t it = 0;
+    int64_t last[P::IS];
+#pragma unroll
+    for (int s = 0; s < P::IS; ++s) last[s] = -1;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
+        const Unit un = decode(u, a, OT);
+        const int32_t y_w = static_cast<int32_t>(un.ot * TILE_O);
+        const int32_t y_qp = static_cast<int32_t>(static_cast<int64_t>(un.g) * a.O + un.ot * TILE_O);
+        for (int64_t kb = 0; kb < nK; ++kb, ++it) {
+            const uint32_t st = it % P::IS;
+            if (!mbar_wait(&in_empty[st], ((it / P::IS) & 1u) ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            uint8_t *dst = in_ring + st * P::IN_STAGE;
+            const int32_t x = static_cast<int32_t>(kb * SLAB_K);
+            mbar_arrive_expect_tx(&in_full[st], bytes);
+            if constexpr (WBF16) {
+                tma_load_2d(dst, &m.w, &in_full[st], x, y_w);
+            } else {
+                tma_load_2d(dst, &m.w, &in_full[st], x, y_w);
+                tma_load_2d(dst + 16384, &m.w, &in_full[st], x + 32, y_w);
+            }
+            tma_load_2d(dst + P::SN_OFF, &m.sn, &in_full[st], x, 2 * un.g);
+            tma_load_2d(dst + P::QP_OFF, &m.qp, &in_full[st],
+                        static_cast<int32_t>(4 * ((kb * SLAB_K) / a.gs)), y_qp);
+#pragma unroll
+            for (int s = 0; s < P::IS; ++s)
+                if (s == static_cast<int>(st)) last[s] = it;
+        }
+    }
+    // Never leave the CTA with a copy still landing in its shared memory.
+#pragma unroll
+    for (int s = 0; s < P::IS; ++s)
+        if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / P::IS) & 1));
+}
+
+// Lane 0 of the TMA warp: X tiles for the MMA.
+template <int XS>
+__device__ __forceinline__ void x_loader(const SearchArgs &a, const CUtensorMap *xmap, int64_t OT,
                                          int64_t U, uint8_t *x_ring, uint64_t *x_full,
                                          uint64_t *x_empty, volatile int *abort_flag) {
     const int64_t nK = a.I / SLAB_K;
@@ -212,12 +268,12 @@ __device__ __forceinline__ void tma_role(const SearchArgs &a, const CUtensorMap 
             }
         }
     }
-    // Never leave the CTA with a copy still landing in its shared memory.
 #pragma unroll
     for (int s = 0; s < XS; ++s)
         if (last[s] >= 0) mbar_wait_drain(&x_full[s], static_cast<uint32_t>((last[s] / XS) & 1));
 }
 
+template <int XS, int AS>
 __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_t U,
                                          uint32_t tmem_base, uint8_t *x_ring, uint8_t *a_ring,
                                          uint64_t *x_full, uint64_t *x_empty, uint64_t *a_full,
@@ -251,8 +307,8 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
 #pragma unroll
                 for (int k = 0; k < SLAB_K / 16; ++k) {
                     umma_f16(tmem_base + static_cast<uint32_t>(h * SUB_N),
-                              sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
-                              IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                             sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
+                             IDESC, (kb > 0 || k > 0) ? 1u : 0u);
                 }
                 umma_commit(&x_empty[xs]);
             }
@@ -299,18 +355,22 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
 
 template <bool WBF16, bool CLAMP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    search_kernel(const __grid_constant__ CUtensorMap xmap, const SearchArgs a) {
+    search_kernel(const __grid_constant__ SearchMaps maps, const SearchArgs a) {
+    using P = Plan<WBF16>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t *x_ring = base;
-    uint8_t *a_ring = base + XS * X_STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(a_ring + AS * A_STAGE_BYTES);
+    uint8_t *a_ring = x_ring + P::XS * X_STAGE_BYTES;
+    uint8_t *in_ring = a_ring + P::AS * A_STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(in_ring + P::IS * P::IN_STAGE);
     uint64_t *x_full = bars;
-    uint64_t *x_empty = x_full + XS;
-    uint64_t *a_full = x_empty + XS;
-    uint64_t *a_empty = a_full + AS;
-    uint64_t *acc_full = a_empty + AS;
+    uint64_t *x_empty = x_full + P::XS;
+    uint64_t *a_full = x_empty + P::XS;
+    uint64_t *a_empty = a_full + P::AS;
+    uint64_t *in_full = a_empty + P::AS;
+    uint64_t *in_empty = in_full + P::IS;
+    uint64_t *acc_full = in_empty + P::IS;
     uint64_t *acc_empty = acc_full + 1;
     uint64_t *drain = acc_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
@@ -322,13 +382,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int64_t U = OT * TB * a.G;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < XS; ++s) {
+        for (int s = 0; s < P::XS; ++s) {
             mbar_init(&x_full[s], 1);
             mbar_init(&x_empty[s], 1);
         }
-        for (int s = 0; s < AS; ++s) {
+        for (int s = 0; s < P::AS; ++s) {
             mbar_init(&a_full[s], NUM_PRODUCER_WARPS * 32);
             mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < P::IS; ++s) {
+            mbar_init(&in_full[s], 1);
+            mbar_init(&in_empty[s], NUM_PRODUCER_WARPS * 32);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4 * 32);
@@ -340,22 +404,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == WARP_TMA && lane == 0) tma_prefetch_desc(&xmap);
+    if (warp == WARP_TMA && lane == 0) {
+        tma_prefetch_desc(&maps.x);
+        tma_prefetch_desc(&maps.w);
+        tma_prefetch_desc(&maps.sn);
+        tma_prefetch_desc(&maps.qp);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp < NUM_PRODUCER_WARPS) {
-        producer_role<WBF16, CLAMP>(a, OT, U, a_ring, a_full, a_empty, abort_flag);
+        producer_role<WBF16, CLAMP>(a, U, in_ring, in_full, in_empty, a_ring, a_full, a_empty,
+                                    abort_flag);
     } else if (warp < WARP_TMA) {
         epilogue_role(a, OT, U, TB, tmem_base, acc_full, acc_empty, abort_flag);
     } else if (warp == WARP_TMA) {
-        if (lane == 0) tma_role(a, &xmap, OT, U, x_ring, x_full, x_empty, abort_flag);
+        if (lane == 0)
+            x_loader<P::XS>(a, &maps.x, OT, U, x_ring, x_full, x_empty, abort_flag);
+        else if (lane == 1)
+            input_loader<WBF16>(a, maps, OT, U, in_ring, in_full, in_empty, abort_flag);
+        __syncwarp();
     } else {
         if (lane == 0)
-            mma_role(a, OT, U, tmem_base, x_ring, a_ring, x_full, x_empty, a_full, a_empty,
-                     acc_full, acc_empty, drain, abort_flag);
+            mma_role<P::XS, P::AS>(a, OT, U, tmem_base, x_ring, a_ring, x_full, x_empty, a_full,
+                                   a_empty, acc_full, acc_empty, drain, abort_flag);
         __syncwarp();
     }
 
@@ -369,15 +443,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 template <bool WBF16, bool CLAMP>
-cudaError_t launch_search_t(const SearchArgs &a, const CUtensorMap &xmap, int num_sms,
+cudaError_t launch_search_t(const SearchArgs &a, const SearchMaps &maps, int num_sms,
                             cudaStream_t st) {
+    constexpr int smem = Plan<WBF16>::SMEM_BYTES;
     static bool attr_set[64] = {};   // per device and template instance
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
         e = cudaFuncSetAttribute(search_kernel<WBF16, CLAMP>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
@@ -385,19 +460,19 @@ cudaError_t launch_search_t(const SearchArgs &a, const CUtensorMap &xmap, int nu
     const int64_t TB = (a.N + TILE_N - 1) / TILE_N;
     const int64_t U = OT * TB * a.G;
     const int grid = static_cast<int>(U < num_sms ? U : num_sms);
-    search_kernel<WBF16, CLAMP><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(xmap, a);
+    search_kernel<WBF16, CLAMP><<<grid, NUM_THREADS, smem, st>>>(maps, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_search(const SearchArgs &a, const CUtensorMap &xmap, int num_sms,
+cudaError_t launch_search(const SearchArgs &a, const SearchMaps &maps, int num_sms,
                           cudaStream_t st) {
     if (a.w_bf16)
-        return a.clamp ? launch_search_t<true, true>(a, xmap, num_sms, st)
-                       : launch_search_t<true, false>(a, xmap, num_sms, st);
-    return a.clamp ? launch_search_t<false, true>(a, xmap, num_sms, st)
-                   : launch_search_t<false, false>(a, xmap, num_sms, st);
+        return a.clamp ? launch_search_t<true, true>(a, maps, num_sms, st)
+                       : launch_search_t<true, false>(a, maps, num_sms, st);
+    return a.clamp ? launch_search_t<false, true>(a, maps, num_sms, st)
+                   : launch_search_t<false, false>(a, maps, num_sms, st);
 }
 
 }  // namespace awq
