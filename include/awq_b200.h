@@ -144,6 +144,26 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
                               int group_size, uint16_t *y, void *stream);
 
 /*
+ * awq_act_stats_noalloc — awq_act_stats without any device allocation.  The
+ * AWQ pages have no counterpart: this exists for callers that cannot allocate
+ * device memory when they compute the statistic (processes that hand nearly
+ * all device memory to their own pool allocator at start-up, or that must not
+ * allocate inside a latency-critical section).  It computes the same values
+ * with the same kernels, but keeps the fp64 chunk partials in a fixed 8 MiB
+ * buffer compiled into the library instead of a temporary allocation, and
+ * calls no allocating routine.
+ * Limit: ceil(N / 128) * in <= 1,048,576; larger calls return
+ * AWQ_ERR_UNSUPPORTED and enqueue nothing.
+ * The first call on a device looks up the buffer's device address (a
+ * cudaGetSymbolAddress call); make that first call before any stream capture.
+ * Every call shares the one buffer per device, so calls whose work overlaps on
+ * the GPU (different streams, or concurrent host threads) race; order them on
+ * one stream.  Arguments and results as for awq_act_stats.  Asynchronous.
+ */
+awq_status_t awq_act_stats_noalloc(const void *X, int x_dtype, int64_t N, int64_t in,
+                                   float clamp_min, float *sX, void *stream);
+
+/*
  * Kernel timing (instrumentation, off by default).  When enabled, each entry
  * point brackets its main kernel launch(es) with CUDA events on `stream`;
  * awq_last_kernel_ms(kind) returns the device time of that kernel in the last

@@ -58,6 +58,8 @@ def _load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.awq_pack_int4.argtypes = [P, I, L, L, P, D, D, I, I, P, P, P, P, P, P]
     lib.awq_linear_w4a16.restype = I
     lib.awq_linear_w4a16.argtypes = [P, L, L, L, P, P, P, P, I, P, P]
+    lib.awq_act_stats_noalloc.restype = I
+    lib.awq_act_stats_noalloc.argtypes = [P, I, L, L, F, P, P]
     lib.awq_set_kernel_timing.restype = None
     lib.awq_set_kernel_timing.argtypes = [I]
     lib.awq_last_kernel_ms.restype = D
@@ -69,7 +71,7 @@ lib = _load_library()
 
 EXPORTS = ("awq_version", "awq_status_string", "awq_last_error", "awq_act_stats",
            "awq_search_layer", "awq_pack_int4", "awq_linear_w4a16", "awq_set_kernel_timing",
-           "awq_last_kernel_ms")
+           "awq_last_kernel_ms", "awq_act_stats_noalloc")
 
 KT_STATS, KT_SEARCH, KT_PACK, KT_APPLY = 0, 1, 2, 3
 

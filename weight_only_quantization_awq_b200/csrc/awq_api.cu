@@ -207,6 +207,8 @@ awq_status_t check_layer(const void *W, int w_dtype, int64_t out, int64_t in, in
 
 }  // namespace
 
+void awq::set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
+
 extern "C" {
 
 int awq_version(void) { return 100; }

@@ -8,6 +8,9 @@
 
 namespace awq {
 
+// Record the calling host thread's last-error text (read back by awq_last_error()).
+void set_last_error(const char *msg);
+
 constexpr int STATS_CHUNK = 128;   // tokens per fp64 partial sum of mean|X|
 constexpr int MAX_GRID = 64;       // grid points per search phase
 
