@@ -289,7 +289,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 11 * args.steps,
+        "gpu_launches": 13 * args.steps,
         "clocks": clk,
         "roofline": {"bound": "tensor", "kernel": "search_kernel",
                      "achieved": round(achieved, 2) if achieved else None,

@@ -431,7 +431,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
     if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 64", (long long)in);
-    if (in > 13312) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld above 13312", (long long)in);
+    if (in > 49152) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld above 49152", (long long)in);
     if (!aligned16(x) || !aligned16(qweight) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
         (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)) || !aligned16(s16) ||
         (reinterpret_cast<uintptr_t>(y) & 1u))

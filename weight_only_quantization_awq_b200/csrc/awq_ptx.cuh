@@ -69,6 +69,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// As mbar_wait, but sleeping between polls: for waits that usually last a
+// whole work unit, so the waiting warps do not take issue slots from the rest.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity,
+                                                volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        __nanosleep(256);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > AWQ_WAIT_CYCLES) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // Same, ignoring the abort flag (used only to drain in-flight copies on exit).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     const long long t0 = clock64();

@@ -10,18 +10,19 @@
 // arithmetic), evaluated for every s = s_X^alpha on the grid.  Neither dW nor E
 // ever reaches global memory.
 //
-// Warp roles (448 threads, one CTA per SM, persistent over work units):
-//   warps 0-7   dW producers: read one slab's inputs (W tile, s and -1/s, group
-//               parameters) from shared memory, form dW for 128 rows x 64
-//               columns, write it as fp16 into shared memory in the
-//               128-byte-swizzled K-major layout the MMA reads, signal a_full.
-//   warps 8-11  epilogue: tcgen05.ld of the 128 x 512 fp32 accumulator (lane =
+// Warp roles (704 threads, one CTA per SM, persistent over work units):
+//   warps 0-15  dW producers (16 columns of one row per thread): read one slab's
+//               inputs (W tile, s and -1/s, group parameters) from shared
+//               memory, form dW for 128 rows x 64 columns, write it as fp16 into
+//               shared memory in the 128-byte-swizzled K-major layout the MMA
+//               reads, signal a_full.
+//   warps 16-19 epilogue: tcgen05.ld of the 128 x 512 fp32 accumulator (lane =
 //               output row), square-and-sum per row, one fp32 partial per
 //               (grid point, token block, row).
-//   warp 12     TMA: lane 0 streams X tiles (256 tokens x 64 channels, fp16
+//   warp 20     TMA: lane 0 streams X tiles (256 tokens x 64 channels, fp16
 //               copy of X scaled by a power of two) into the X ring; lane 1
 //               streams each slab's producer inputs into the input ring.
-//   warp 13     MMA: allocates 512 TMEM columns; one thread issues
+//   warp 21     MMA: allocates 512 TMEM columns; one thread issues
 //               tcgen05.mma M=128 N=256 K=16 (two N=256 halves per slab) and
 //               tcgen05.commit releases ring stages and the accumulator.
 // Work units are (g fastest, then output tile, then token block) and are dealt
@@ -36,10 +37,11 @@ namespace awq {
 
 namespace {
 
-constexpr int NUM_PRODUCER_WARPS = 8;
-constexpr int WARP_TMA = 12;
-constexpr int WARP_MMA = 13;
-constexpr int NUM_THREADS = 14 * 32;
+constexpr int NUM_PRODUCER_WARPS = 16;
+constexpr int EPI_WARP0 = 16;                          // warps 16-19: TMEM lane quadrants 0-3
+constexpr int WARP_TMA = 20;
+constexpr int WARP_MMA = 21;
+constexpr int NUM_THREADS = 22 * 32;
 constexpr int X_STAGE_BYTES = SUB_N * SLAB_K * 2;      // 32 KB of fp16 X
 constexpr int A_STAGE_BYTES = TILE_O * SLAB_K * 2;     // 16 KB of fp16 dW
 constexpr uint32_t TMEM_COLS = 512;
@@ -144,10 +146,11 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
                                               uint64_t *a_full, uint64_t *a_empty,
                                               volatile int *abort_flag) {
     using P = Plan<WBF16>;
-    const int t = threadIdx.x;          // 0..255
-    const int r = t >> 1, hc = t & 1;   // row in tile, half of the 64-wide slab
+    const int t = threadIdx.x;          // 0..511
+    const int r = t >> 2, qc = t & 3;   // row in tile, 16-column quarter of the 64-wide slab
+    const int lane = t & 31;
     const int gps = a.gs == 32 ? 2 : 1; // group-parameter entries per row in a stage
-    const int jq = a.gs == 32 ? hc : 0; // this thread's entry
+    const int jq = a.gs == 32 ? (qc >> 1) : 0;
     const int64_t nK = a.I / SLAB_K;
     uint32_t it = 0;
     for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
@@ -158,12 +161,16 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
             const uint8_t *in = in_ring + is * P::IN_STAGE;
             uint8_t *dst = a_ring + as * A_STAGE_BYTES;
             const float4 prm = reinterpret_cast<const float4 *>(in + P::QP_OFF)[r * gps + jq];
-            const float *s_sm = reinterpret_cast<const float *>(in + P::SN_OFF) + hc * 32;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int cc = 0; cc < 2; ++cc) {
+                // Quarters 2-3 take their two 8-column chunks in the opposite order, so
+                // the s / -1/s loads of one warp instruction never share banks.
+                const int c = cc ^ (qc >> 1);
+                const int ch = qc * 2 + c;                 // 16-byte chunk within the 128-byte row
+                const float *s_sm = reinterpret_cast<const float *>(in + P::SN_OFF) + ch * 8;
                 float w[8];
                 if constexpr (WBF16) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(in + sw128_offset(r, hc * 4 + c));
+                    const uint4 v = *reinterpret_cast<const uint4 *>(in + sw128_offset(r, ch));
                     const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -171,22 +178,28 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
                         w[2 * k + 1] = __uint_as_float(u4[k] & 0xFFFF0000u);
                     }
                 } else {
-                    const uint8_t *sub = in + hc * 16384;   // columns hc*32 .. hc*32+31
-                    const float4 v0 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, 2 * c));
-                    const float4 v1 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, 2 * c + 1));
+                    const uint8_t *sub = in + (ch >> 2) * 16384;   // 32-column fp32 sub-tile
+                    const int sc = (ch & 3) * 2;                     // its 16-byte chunks
+                    const float4 v0 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, sc));
+                    const float4 v1 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, sc + 1));
                     w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
                     w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
                 }
-                const float4 s0 = *reinterpret_cast<const float4 *>(s_sm + 8 * c);
-                const float4 s1 = *reinterpret_cast<const float4 *>(s_sm + 8 * c + 4);
-                const float4 n0 = *reinterpret_cast<const float4 *>(s_sm + 64 + 8 * c);
-                const float4 n1 = *reinterpret_cast<const float4 *>(s_sm + 64 + 8 * c + 4);
-                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, hc * 4 + c)) =
+                const float4 s0 = *reinterpret_cast<const float4 *>(s_sm);
+                const float4 s1 = *reinterpret_cast<const float4 *>(s_sm + 4);
+                const float4 n0 = *reinterpret_cast<const float4 *>(s_sm + 64);
+                const float4 n1 = *reinterpret_cast<const float4 *>(s_sm + 68);
+                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, ch)) =
                     dw_chunk8<CLAMP>(w, s0, s1, n0, n1, prm);
             }
-            mbar_arrive(&in_empty[is]);
+            // One arrival per warp: every lane's reads and fenced writes are ordered
+            // before lane 0's arrive by the warp barrier.
             fence_proxy_async_smem();
-            mbar_arrive(&a_full[as]);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&in_empty[is]);
+                mbar_arrive(&a_full[as]);
+            }
         }
     }
 }
@@ -333,7 +346,7 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
     uint32_t accit = 0;
     for (int64_t u = blockIdx.x; u < U; u += gridDim.x, ++accit) {
         const Unit un = decode(u, a, OT);
-        const bool ok = mbar_wait(acc_full, accit & 1u, abort_flag);
+        const bool ok = mbar_wait_sleep(acc_full, accit & 1u, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) return;
         tc_fence_after();
         float sum = 0.0f;
@@ -387,12 +400,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&x_empty[s], 1);
         }
         for (int s = 0; s < P::AS; ++s) {
-            mbar_init(&a_full[s], NUM_PRODUCER_WARPS * 32);
+            mbar_init(&a_full[s], NUM_PRODUCER_WARPS);
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < P::IS; ++s) {
             mbar_init(&in_full[s], 1);
-            mbar_init(&in_empty[s], NUM_PRODUCER_WARPS * 32);
+            mbar_init(&in_empty[s], NUM_PRODUCER_WARPS);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4 * 32);
@@ -418,7 +431,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (warp < NUM_PRODUCER_WARPS) {
         producer_role<WBF16, CLAMP>(a, U, in_ring, in_full, in_empty, a_ring, a_full, a_empty,
                                     abort_flag);
-    } else if (warp < WARP_TMA) {
+    } else if (warp < EPI_WARP0 + 4) {
         epilogue_role(a, OT, U, TB, tmem_base, acc_full, acc_empty, abort_flag);
     } else if (warp == WARP_TMA) {
         if (lane == 0)
