@@ -41,9 +41,9 @@ ROTATE = 3
 APPLY_M = 1
 
 # DRAM traffic of one search-kernel launch on this workload, from the ncu capture
-# summarised in profiles/search_kernel_attn_proj_4096.md, valid only for the
+# summarised in profiles/search_kernel_attn_proj_4096x4096_n4096.md, valid only for the
 # kernel source it was taken on (sha256 of csrc/k_search.cu, first 16 hex).
-SEARCH_TRAFFIC = {"source_sha": None, "bytes": None}
+SEARCH_TRAFFIC = {"source_sha": "f07af1a0ea671b9c", "bytes": 353965568}
 
 
 def _env_int(k, d):

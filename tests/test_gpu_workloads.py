@@ -1,0 +1,125 @@
+"""Full-size parity for the larger workloads (GPU search at full size, oracle
+on seeded row samples; every INT4 code of the chosen quantisation checked
+bit-exact against the oracle's packing).
+
+  workload 3: Llama-7B MLP, gate||up searched jointly (22016 x 4096) and down
+              (4096 x 11008), N = 8192 Student-t(4) tokens, symmetric;
+  workload 4: Llama-13B up_proj 13824 x 5120, N = 65536, asymmetric; the
+              oracle evaluates the loss at alpha in {0, 0.5} on sampled rows
+              below 1024, codes are checked at the GPU-chosen alpha;
+  workload 5: Llama-7B block linear o (4096 x 4096) and down (4096 x 11008),
+              N = 16384, asymmetric with the 11-point clip grid after alpha*.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from synthetic import ALPHA_GRID, CLIP_GRID
+
+pytestmark = pytest.mark.gpu
+
+ROW_RTOL = 2e-3
+TIE_RTOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def awq():
+    import weight_only_quantization_awq_b200 as m
+    assert torch.cuda.is_available()
+    return m
+
+
+def dev(a):
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def sample_rows(O, k, seed, below=None):
+    hi = O if below is None else min(O, below)
+    r = np.random.default_rng(seed).choice(hi, size=k - 2, replace=False)
+    return np.unique(np.concatenate([[0, hi - 1], r])).astype(np.int64)
+
+
+def check_rows(lr_gpu, ref_rows, rows):
+    np.testing.assert_allclose(lr_gpu[:, rows], ref_rows, rtol=ROW_RTOL)
+
+
+def check_codes(awq, W, Wd, sXd, alpha, clip, qt):
+    got = awq.awq_pack_int4(Wd, sXd, alpha, clip, 128, qt)
+    ref = oracle.pack_int4(W, sXd.cpu().numpy(), alpha, clip, 128, qt)
+    assert np.array_equal(got["qweight"].cpu().numpy().view(np.uint32), ref["qweight"])
+    assert np.array_equal(got["scales"].cpu().numpy().view(np.uint16), ref["scales"])
+    if qt == 1:
+        assert np.array_equal(got["zeros"].cpu().numpy().view(np.uint32), ref["zeros"])
+
+
+def run_layer(awq, wid, layer, qt, rows_k, clip=None, seed=0):
+    W = synthetic.layer_weights(wid, layer)
+    X = synthetic.layer_activations(wid, layer)
+    Wd, Xd = dev(W), dev(X)
+    sXd = awq.awq_act_stats(Xd)
+    sX = sXd.cpu().numpy()
+    assert np.array_equal(sX, oracle.act_stats(X))
+    got = awq.awq_search_layer(Wd, Xd, sXd, 128, 4, qt, ALPHA_GRID, clip=clip, loss_row=True)
+    lr = got["loss_row"].cpu().numpy().astype(np.float64)
+    O = W.shape[0]
+    rows = sample_rows(O, rows_k, seed)
+    return W, X, Wd, Xd, sXd, sX, got, lr, rows
+
+
+def test_workload3_gate_up_joint(awq):
+    W, X, Wd, Xd, sXd, sX, got, lr, rows = run_layer(awq, 3, "gate_up", 0, 12, seed=31)
+    assert W.shape == (22016, 4096)
+    ref = oracle.search_layer(W, X, sX, 128, 0, ALPHA_GRID, rows=rows)
+    check_rows(lr, ref["loss_row"], rows)
+    np.testing.assert_allclose(got["loss"], lr.sum(axis=1) / (X.shape[0] * W.shape[0]), rtol=1e-6)
+    assert got["best_alpha"] == int(np.argmin(got["loss"]))
+    check_codes(awq, W, Wd, sXd, float(ALPHA_GRID[got["best_alpha"]]), 1.0, 0)
+
+
+def test_workload3_down(awq):
+    W, X, Wd, Xd, sXd, sX, got, lr, rows = run_layer(awq, 3, "down", 0, 10, seed=32)
+    assert W.shape == (4096, 11008)
+    ref = oracle.search_layer(W, X, sX, 128, 0, ALPHA_GRID, rows=rows)
+    check_rows(lr, ref["loss_row"], rows)
+    check_codes(awq, W, Wd, sXd, float(ALPHA_GRID[got["best_alpha"]]), 1.0, 0)
+
+
+def test_workload4_up_proj_asym(awq):
+    W = synthetic.layer_weights(4, "up_proj")
+    X = synthetic.layer_activations(4, "up_proj")
+    assert W.shape == (13824, 5120) and X.shape == (65536, 5120)
+    Wd, Xd = dev(W), dev(X)
+    sXd = awq.awq_act_stats(Xd)
+    sX = sXd.cpu().numpy()
+    assert np.array_equal(sX, oracle.act_stats(X))
+    got = awq.awq_search_layer(Wd, Xd, sXd, 128, 4, 1, ALPHA_GRID, loss_row=True)
+    lr = got["loss_row"].cpu().numpy().astype(np.float64)
+    rows = sample_rows(13824, 8, 41, below=1024)
+    ref = oracle.search_layer(W, X, sX, 128, 1, np.array([0.0, 0.5]), rows=rows)
+    check_rows(lr[[0, 10]], ref["loss_row"], rows)
+    # alpha* itself is not evaluated by the oracle here: check it is the GPU's own argmin,
+    # and that the codes at it are the oracle's.
+    assert got["best_alpha"] == int(np.argmin(got["loss"]))
+    del Xd
+    torch.cuda.empty_cache()
+    check_codes(awq, W, Wd, sXd, float(ALPHA_GRID[got["best_alpha"]]), 1.0, 1)
+
+
+@pytest.mark.parametrize("layer", ["o", "down"])
+def test_workload5_asym_with_clip(awq, layer):
+    W, X, Wd, Xd, sXd, sX, got, lr, rows = run_layer(awq, 5, layer, 1, 6, clip=CLIP_GRID,
+                                                     seed=51)
+    G = len(ALPHA_GRID)
+    ref = oracle.search_layer(W, X, sX, 128, 1, ALPHA_GRID, rows=rows)
+    check_rows(lr[:G], ref["loss_row"], rows)
+    # the clip phase at the GPU's alpha*
+    a_star = ALPHA_GRID[[got["best_alpha"]]]
+    ref2 = oracle.search_layer(W, X, sX, 128, 1, a_star, clip=CLIP_GRID, rows=rows)
+    check_rows(lr[G:], ref2["loss_row"][1:], rows)
+    assert got["loss"][G] == pytest.approx(got["loss"][got["best_alpha"]], rel=1e-12)
+    assert got["best_clip"] == int(np.argmin(got["loss"][G:]))
+    check_codes(awq, W, Wd, sXd, float(a_star[0]), float(CLIP_GRID[got["best_clip"]]), 1)
