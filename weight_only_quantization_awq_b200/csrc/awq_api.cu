@@ -131,8 +131,8 @@ awq_status_t make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, size_t elem, 
 //   x  : fp16 copy of X [N, I], boxes of 64 channels x 256 tokens, 128B swizzle;
 //   w  : W [O, I], 128 rows x 128 bytes per box, 128B swizzle;
 //   sn : scale table [2G, I] fp32, boxes of 64 channels x (s row, -1/s row);
-//   qp : group parameters [G*O, 4*I/gs] fp32, boxes of 128 rows x the groups
-//        one 64-column slab touches.
+//   qp : group parameters [G * I/gs][O][4] fp32 (3-D), boxes of 128 rows x the
+//        groups one 64-column slab touches.
 awq_status_t make_search_maps(awq::SearchMaps *m, const uint16_t *x16, int64_t N, const void *W,
                               bool w_bf16, int64_t O, int64_t I, const float *sn,
                               const float4 *qparam, int G, int gs) {
@@ -147,10 +147,18 @@ awq_status_t make_search_maps(awq::SearchMaps *m, const uint16_t *x16, int64_t N
     if (awq_status_t s = make_map_2d(&m->sn, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, sn, I, 2 * G,
                                      awq::SLAB_K, 2, CU_TENSOR_MAP_SWIZZLE_NONE))
         return s;
-    const int gps = gs == 32 ? 2 : 1;
-    return make_map_2d(&m->qp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, qparam, 4 * (I / gs),
-                       static_cast<uint64_t>(G) * O, 4 * gps, awq::TILE_O,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    auto enc = get_encode();
+    if (!enc) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+    const cuuint32_t gps = gs == 32 ? 2 : 1;
+    cuuint64_t dims[3] = {4, static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(G) * (I / gs)};
+    cuuint64_t strides[2] = {16, static_cast<cuuint64_t>(O) * 16};
+    cuuint32_t box[3] = {4, static_cast<cuuint32_t>(awq::TILE_O), gps};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(&m->qp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float4 *>(qparam), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(AWQ_ERR_CUDA, "cuTensorMapEncodeTiled (qp) failed (%d)", (int)r);
+    return AWQ_OK;
 }
 
 bool valid_dtype(int d) { return d == AWQ_F32 || d == AWQ_BF16; }
@@ -303,6 +311,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     size_t bytes = 0;
     bytes += Workspace::up(sizeof(uint16_t) * N * in);
     bytes += Workspace::up(sizeof(float) * 2 * G * in);
+    bytes += Workspace::up(awq::scale_scratch_bytes(G, in));
     bytes += Workspace::up(sizeof(float4) * G * out * nG);
     bytes += Workspace::up(sizeof(float) * G * TB * out);
     bytes += Workspace::up(sizeof(double) * Gtot);
@@ -312,6 +321,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     if (awq_status_t s = ws.reserve(bytes)) return s;
     uint16_t *x16 = ws.take<uint16_t>(N * in);
     float *sn = ws.take<float>(2 * G * in);
+    char *sc_scratch = ws.take<char>(awq::scale_scratch_bytes(G, in));
     float4 *qparam = ws.take<float4>(G * out * nG);
     float *part = ws.take<float>(G * TB * out);
     double *loss_d = ws.take<double>(Gtot);
@@ -338,7 +348,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
         ap.value[k] = alpha[k];
         cp.value[k] = 1.0;
     }
-    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, sn, st));
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, sn, sc_scratch, st));
     AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM, sn,
                                       cp, n_alpha, qparam, st));
     a.G = n_alpha;
@@ -358,7 +368,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
     if (n_clip > 0) {
         awq::GridParams cp2{};
         for (int k = 0; k < n_clip; ++k) cp2.value[k] = clip[k];
-        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, sn, st));
+        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, sn, sc_scratch, st));
         AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM,
                                           sn, cp2, n_clip, qparam, st));
         a.G = n_clip;
@@ -406,11 +416,14 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, 
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     Workspace ws(st);
-    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(float) * 2 * in))) return s;
+    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(float) * 2 * in) +
+                                    Workspace::up(awq::scale_scratch_bytes(1, in))))
+        return s;
     float *sn = ws.take<float>(2 * in);   // row 0: s, row 1: -1/s
+    char *sc_scratch = ws.take<char>(awq::scale_scratch_bytes(1, in));
     awq::GridParams ap{};
     ap.value[0] = alpha;
-    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, sn, st));
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, sn, sc_scratch, st));
     const int64_t nG = in / group_size;
     if (zeros) AWQ_CUDA(cudaMemsetAsync(zeros, 0, sizeof(uint32_t) * out * ((nG + 7) / 8), st));
     kt_reset(2);

@@ -36,10 +36,13 @@ cudaError_t launch_x_to_f16(const void *X, bool x_bf16, int64_t n, unsigned *max
 // ---- scale table sn[G][2][I]: row 2g holds s_g, row 2g+1 holds -1/s_g.
 // alpha.value[g] is grid point g's alpha; if best_idx != nullptr every row uses
 // alpha.value[*best_idx] instead (the second, clip phase).
+// scratch: scale_scratch_bytes(G, I) bytes of device workspace.
+int64_t scale_scratch_bytes(int G, int64_t I);
 cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
-                               const int *best_idx, float *sn, cudaStream_t st);
+                               const int *best_idx, float *sn, void *scratch, cudaStream_t st);
 
-// ---- per-(grid point, row, group) quantiser parameters {Delta, 1/Delta, -qhi, -qlo}
+// ---- per-(grid point, group, row) quantiser parameters {Delta, 1/Delta, -qhi, -qlo},
+// layout qparam[g][group][row] (rows fastest)
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
                                 bool asym, const float *sn, const GridParams &clip, int G,
                                 float4 *qparam, cudaStream_t st);
@@ -49,7 +52,7 @@ cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I
 //   x  : fp16 copy of X [N, I], box 64 x 256, 128B swizzle
 //   w  : W [O, I] (bf16: box 64 x 128; fp32: box 32 x 128), 128B swizzle
 //   sn : scale table [2G, I] fp32, box 64 x 2
-//   qp : group parameters [G*O, 4*I/gs] fp32, box (4 * groups per slab) x 128
+//   qp : group parameters [G * I/gs][O][4] fp32 (3-D), box 4 x 128 rows x groups per slab
 struct SearchMaps {
     CUtensorMap x, w, sn, qp;
 };

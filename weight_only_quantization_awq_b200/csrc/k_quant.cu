@@ -18,34 +18,60 @@
 namespace awq {
 
 // ------------------------------------------------------------ scale table
-__global__ void __launch_bounds__(256) scale_table_kernel(const float *__restrict__ sX, int64_t I,
-                                                          GridParams alpha,
-                                                          const int *__restrict__ best_idx,
-                                                          float *__restrict__ sn) {
+// Pass 1: t[g][i] = pow(s_X[i], alpha_g) in fp64, and max_i t[g][i] through an
+// atomic max on the bit patterns (t >= 0, so bit order is value order).
+// Pass 2: s = fp32(t / max), -1/s.
+__global__ void __launch_bounds__(256) scale_pow_kernel(const float *__restrict__ sX, int64_t I,
+                                                        GridParams alpha,
+                                                        const int *__restrict__ best_idx,
+                                                        double *__restrict__ t,
+                                                        unsigned long long *__restrict__ max_bits) {
     __shared__ double red[256];
-    const int g = blockIdx.x;
+    const int g = blockIdx.y;
     const double a = best_idx ? alpha.value[*best_idx] : alpha.value[g];
-    double m = 0.0;
-    for (int64_t i = threadIdx.x; i < I; i += blockDim.x)
-        m = fmax(m, pow(static_cast<double>(sX[i]), a));
-    red[threadIdx.x] = m;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    double v = 0.0;
+    if (i < I) {
+        v = pow(static_cast<double>(sX[i]), a);
+        t[g * I + i] = v;
+    }
+    red[threadIdx.x] = v;
     __syncthreads();
     for (int off = 128; off > 0; off >>= 1) {
         if (threadIdx.x < off) red[threadIdx.x] = fmax(red[threadIdx.x], red[threadIdx.x + off]);
         __syncthreads();
     }
-    m = red[0];
-    for (int64_t i = threadIdx.x; i < I; i += blockDim.x) {
-        const double t = pow(static_cast<double>(sX[i]), a);
-        const float s = __double2float_rn(__ddiv_rn(t, m));
-        sn[(2 * g) * I + i] = s;
-        sn[(2 * g + 1) * I + i] = -__frcp_rn(s);
-    }
+    if (threadIdx.x == 0)
+        atomicMax(&max_bits[g], static_cast<unsigned long long>(__double_as_longlong(red[0])));
+}
+
+__global__ void __launch_bounds__(256) scale_div_kernel(const double *__restrict__ t, int64_t I,
+                                                        const unsigned long long *__restrict__ max_bits,
+                                                        float *__restrict__ sn) {
+    const int g = blockIdx.y;
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= I) return;
+    const double m = __longlong_as_double(static_cast<long long>(max_bits[g]));
+    const float s = __double2float_rn(__ddiv_rn(t[g * I + i], m));
+    sn[(2 * g) * I + i] = s;
+    sn[(2 * g + 1) * I + i] = -__frcp_rn(s);
+}
+
+int64_t scale_scratch_bytes(int G, int64_t I) {
+    return static_cast<int64_t>(G) * I * 8 + static_cast<int64_t>(G) * 8;
 }
 
 cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alpha, int G,
-                               const int *best_idx, float *sn, cudaStream_t st) {
-    scale_table_kernel<<<G, 256, 0, st>>>(sX, I, alpha, best_idx, sn);
+                               const int *best_idx, float *sn, void *scratch, cudaStream_t st) {
+    double *t = static_cast<double *>(scratch);
+    unsigned long long *mb = reinterpret_cast<unsigned long long *>(t + static_cast<int64_t>(G) * I);
+    cudaError_t e = cudaMemsetAsync(mb, 0, sizeof(unsigned long long) * G, st);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>((I + 255) / 256), static_cast<unsigned>(G));
+    scale_pow_kernel<<<grid, 256, 0, st>>>(sX, I, alpha, best_idx, t, mb);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    scale_div_kernel<<<grid, 256, 0, st>>>(t, I, mb, sn);
     return cudaGetLastError();
 }
 
@@ -60,82 +86,88 @@ __device__ __forceinline__ float safe_rcp(float d) {
     return isinf(r) ? 3.4028234663852886e38f : r;
 }
 
-// One warp per (row, group); each lane holds gs/32 elements of the group and
-// loops over the G grid points, so W is read once for all of them.
-template <bool WBF16, int EPL>
-__global__ void __launch_bounds__(256) group_params_kernel(
-    const void *__restrict__ W, int64_t O, int64_t I, int gs, bool asym,
-    const float *__restrict__ sn, GridParams clip, int G, float4 *__restrict__ qparam) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t nG = I / gs;
-    const int64_t pair = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-    if (pair >= O * nG) return;
-    const int64_t o = pair / nG, j = pair % nG;
-    const int64_t col = j * gs + static_cast<int64_t>(lane) * EPL;
-    float w[EPL];
+// One thread per (row, group): the thread keeps its group's gs weights in
+// registers and loops over the G grid points; each grid point's s values for
+// the group are broadcast from shared memory.  Output layout qparam[g][j][o]
+// (rows fastest) so the writes coalesce.
+template <bool WBF16, int GS>
+__global__ void __launch_bounds__(128) group_params_kernel(
+    const void *__restrict__ W, int64_t O, int64_t I, bool asym, const float *__restrict__ sn,
+    GridParams clip, int G, float4 *__restrict__ qparam) {
+    __shared__ __align__(16) float s_sm[MAX_GRID][GS];
+    const int64_t j = blockIdx.y;
+    const int64_t nG = I / GS;
+    for (int k = threadIdx.x; k < G * GS; k += blockDim.x)
+        s_sm[k / GS][k % GS] = sn[static_cast<int64_t>(2 * (k / GS)) * I + j * GS + (k % GS)];
+    __syncthreads();
+    const int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (o >= O) return;
+    constexpr int NW = WBF16 ? GS / 2 : GS;      // 32-bit words of the group
+    uint32_t wr[NW];
+    const uint4 *src = WBF16 ? reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(W) + o * I + j * GS)
+                             : reinterpret_cast<const uint4 *>(static_cast<const float *>(W) + o * I + j * GS);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-        if constexpr (WBF16) {
-            const uint16_t b = static_cast<const uint16_t *>(W)[o * I + col + e];
-            w[e] = __uint_as_float(static_cast<uint32_t>(b) << 16);
-        } else {
-            w[e] = static_cast<const float *>(W)[o * I + col + e];
-        }
+    for (int k = 0; k < NW / 4; ++k) {
+        const uint4 v = __ldg(src + k);
+        wr[4 * k] = v.x; wr[4 * k + 1] = v.y; wr[4 * k + 2] = v.z; wr[4 * k + 3] = v.w;
     }
     for (int g = 0; g < G; ++g) {
-        const float *s = sn + static_cast<int64_t>(2 * g) * I + col;
         float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-            const float wp = __fmul_rn(w[e], s[e]);
-            mx = fmaxf(mx, wp);
-            mn = fminf(mn, wp);
-            amax = fmaxf(amax, fabsf(wp));
-        }
+        for (int e4 = 0; e4 < GS / 4; ++e4) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(&s_sm[g][4 * e4]);
+            const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-        }
-        if (lane == 0) {
-            const double r = clip.value[g];
-            float D, qlo, qhi;
-            if (!asym) {
-                D = __fdiv_rn(clip_bound(amax, r), 7.0f);
-                qlo = -8.0f;
-                qhi = 7.0f;
-            } else {
-                const float hi = clip_bound(mx, r), lo = clip_bound(mn, r);
-                D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
-                float z = 0.0f;
-                if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
-                qlo = -z;
-                qhi = 15.0f - z;
-                if (D == 0.0f) qhi = 0.0f;
+            for (int k = 0; k < 4; ++k) {
+                const int e = 4 * e4 + k;
+                float w;
+                if constexpr (WBF16)
+                    w = (e & 1) ? __uint_as_float(wr[e >> 1] & 0xFFFF0000u) : __uint_as_float(wr[e >> 1] << 16);
+                else
+                    w = __uint_as_float(wr[e]);
+                const float wp = __fmul_rn(w, sv[k]);
+                if (asym) {
+                    mx = fmaxf(mx, wp);
+                    mn = fminf(mn, wp);
+                } else {
+                    amax = fmaxf(amax, fabsf(wp));
+                }
             }
-            // {Delta, 1/Delta, -qhi, -qlo}: the search kernel works with -q.
-            qparam[(static_cast<int64_t>(g) * O + o) * nG + j] =
-                make_float4(D, safe_rcp(D), -qhi, -qlo);
         }
+        const double r = clip.value[g];
+        float D, qlo, qhi;
+        if (!asym) {
+            D = __fdiv_rn(clip_bound(amax, r), 7.0f);
+            qlo = -8.0f;
+            qhi = 7.0f;
+        } else {
+            const float hi = clip_bound(mx, r), lo = clip_bound(mn, r);
+            D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+            float z = 0.0f;
+            if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+            qlo = -z;
+            qhi = 15.0f - z;
+            if (D == 0.0f) qhi = 0.0f;
+        }
+        // {Delta, 1/Delta, -qhi, -qlo}: the search kernel works with -q.
+        qparam[(static_cast<int64_t>(g) * nG + j) * O + o] = make_float4(D, safe_rcp(D), -qhi, -qlo);
     }
 }
 
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
                                 bool asym, const float *sn, const GridParams &clip, int G,
                                 float4 *qparam, cudaStream_t st) {
-    const int64_t pairs = O * (I / gs);
-    const unsigned blocks = static_cast<unsigned>((pairs + 7) / 8);
-#define AWQ_GP(WB, E) \
-    group_params_kernel<WB, E><<<blocks, 256, 0, st>>>(W, O, I, gs, asym, sn, clip, G, qparam)
+    const dim3 grid(static_cast<unsigned>((O + 127) / 128), static_cast<unsigned>(I / gs));
+#define AWQ_GP(WB, GSZ) \
+    group_params_kernel<WB, GSZ><<<grid, 128, 0, st>>>(W, O, I, asym, sn, clip, G, qparam)
     if (w_bf16) {
-        if (gs == 32) AWQ_GP(true, 1);
-        else if (gs == 64) AWQ_GP(true, 2);
-        else AWQ_GP(true, 4);
+        if (gs == 32) AWQ_GP(true, 32);
+        else if (gs == 64) AWQ_GP(true, 64);
+        else AWQ_GP(true, 128);
     } else {
-        if (gs == 32) AWQ_GP(false, 1);
-        else if (gs == 64) AWQ_GP(false, 2);
-        else AWQ_GP(false, 4);
+        if (gs == 32) AWQ_GP(false, 32);
+        else if (gs == 64) AWQ_GP(false, 64);
+        else AWQ_GP(false, 128);
     }
 #undef AWQ_GP
     return cudaGetLastError();
@@ -207,27 +239,37 @@ __global__ void __launch_bounds__(256) pack_kernel(const void *__restrict__ W, i
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
         }
         float D, z = 0.0f;
-        uint32_t word = 0;
         if (!asym) {
             const float a = clip == 1.0 ? amax : __double2float_rn(__dmul_rn((double)amax, clip));
             D = __fdiv_rn(a, 7.0f);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                float q = 0.0f;
-                if (D != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(wp[k], D)), -8.0f), 7.0f);
-                word |= (static_cast<uint32_t>(static_cast<int>(q) + 8) & 0xFu) << (4 * k);
-            }
         } else {
             const float hi = clip == 1.0 ? mx : __double2float_rn(__dmul_rn((double)mx, clip));
             const float lo = clip == 1.0 ? mn : __double2float_rn(__dmul_rn((double)mn, clip));
             D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
             if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+        }
+        // q = rint(RN(W'/Delta)) from the reciprocal product W' * RN(1/Delta): every
+        // decision that survives the clamp has |W'/Delta| <= 15.5, where the product
+        // is within 2^-19 of RN(W'/Delta); products within 2^-16 of a half-integer
+        // (exact ties included) are redone with the correctly rounded division.
+        float q[8];
+        const float invD = D != 0.0f ? __frcp_rn(D) : 0.0f;
+        bool near_tie = false;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                float q = 0.0f;
-                if (D != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(wp[k], D)) + z, 0.0f), 15.0f);
-                word |= (static_cast<uint32_t>(static_cast<int>(q)) & 0xFu) << (4 * k);
-            }
+        for (int k = 0; k < 8; ++k) {
+            q[k] = __fsub_rn(__fmaf_rn(wp[k], invD, 12582912.0f), 12582912.0f);
+            near_tie |= fabsf(__fmaf_rn(wp[k], invD, -q[k])) > 0.5f - 1.0f / 65536.0f;
+        }
+        if (near_tie && D != 0.0f) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) q[k] = rintf(__fdiv_rn(wp[k], D));
+        }
+        uint32_t word = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float c = asym ? fminf(fmaxf(q[k] + z, 0.0f), 15.0f)
+                                 : fminf(fmaxf(q[k], -8.0f), 7.0f) + 8.0f;
+            word |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * k);
         }
         if (!active) continue;
         qweight[idx] = word;

@@ -49,7 +49,7 @@ constexpr uint32_t IDESC = idesc_f16_f32(TILE_O, SUB_N, false);
 constexpr float MAGIC = 12582912.0f;                   // 1.5 * 2^23: x + MAGIC - MAGIC = rint(x)
 
 // Shared-memory plan, per weight type.  Input stage = W tile, then s / -1/s of
-// the slab (2 x 64 fp32), then the 128 rows' group parameters (1 or 2 float4).
+// the slab (2 x 64 fp32), then the group parameters [1 or 2 groups][128 rows] float4.
 template <bool WBF16>
 struct Plan {
     static constexpr int XS = WBF16 ? 4 : 3;            // X ring stages
@@ -84,8 +84,10 @@ __device__ __forceinline__ Unit decode(int64_t u, const SearchArgs &a, int64_t O
 }
 
 // Distance from a half-integer below which the reciprocal product may round to
-// a different code than the correctly rounded quotient: |W'/Delta| <= 32, so
-// W' * RN(1/Delta) and RN(W'/Delta) differ by at most 32 * 2^-23 = 2^-18.
+// a different code than the correctly rounded quotient.  Every rounding
+// decision that survives the code clamp has |W'/Delta| <= 15.5 (codes span at
+// most 16 levels around 0), where W' * RN(1/Delta) and RN(W'/Delta) differ by at
+// most 16 * 2^-23 = 2^-19; beyond that both sides saturate to the same code.
 constexpr float TIE_BAND = 0.5f - 1.0f / 65536.0f;
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
@@ -149,8 +151,7 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
     const int t = threadIdx.x;          // 0..511
     const int r = t >> 2, qc = t & 3;   // row in tile, 16-column quarter of the 64-wide slab
     const int lane = t & 31;
-    const int gps = a.gs == 32 ? 2 : 1; // group-parameter entries per row in a stage
-    const int jq = a.gs == 32 ? (qc >> 1) : 0;
+    const int jq = a.gs == 32 ? (qc >> 1) : 0;   // which of the slab's groups (stage holds [groups][128 rows])
     const int64_t nK = a.I / SLAB_K;
     uint32_t it = 0;
     for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
@@ -160,7 +161,7 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
             if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag)) return;
             const uint8_t *in = in_ring + is * P::IN_STAGE;
             uint8_t *dst = a_ring + as * A_STAGE_BYTES;
-            const float4 prm = reinterpret_cast<const float4 *>(in + P::QP_OFF)[r * gps + jq];
+            const float4 prm = reinterpret_cast<const float4 *>(in + P::QP_OFF)[jq * TILE_O + r];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 // Quarters 2-3 take their two 8-column chunks in the opposite order, so
@@ -221,7 +222,7 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
     for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
         const Unit un = decode(u, a, OT);
         const int32_t y_w = static_cast<int32_t>(un.ot * TILE_O);
-        const int32_t y_qp = static_cast<int32_t>(static_cast<int64_t>(un.g) * a.O + un.ot * TILE_O);
+        const int64_t nG = a.I / a.gs;
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
             const uint32_t st = it % P::IS;
             if (!mbar_wait(&in_empty[st], ((it / P::IS) & 1u) ^ 1u, abort_flag)) {
@@ -238,8 +239,8 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
                 tma_load_2d(dst + 16384, &m.w, &in_full[st], x + 32, y_w);
             }
             tma_load_2d(dst + P::SN_OFF, &m.sn, &in_full[st], x, 2 * un.g);
-            tma_load_2d(dst + P::QP_OFF, &m.qp, &in_full[st],
-                        static_cast<int32_t>(4 * ((kb * SLAB_K) / a.gs)), y_qp);
+            tma_load_3d(dst + P::QP_OFF, &m.qp, &in_full[st], 0, y_w,
+                        static_cast<int32_t>(static_cast<int64_t>(un.g) * nG + (kb * SLAB_K) / a.gs));
 #pragma unroll
             for (int s = 0; s < P::IS; ++s)
                 if (s == static_cast<int>(st)) last[s] = it;

@@ -1,9 +1,9 @@
 // Activation statistic s_X[i] = mean_n |X[n, i]| (AWQ guide, section 三, step 1;
 // paper summary, Method: s_X is the per-channel activation magnitude).
 //
-// HBM-bound column reduction.  Phase 1: each thread owns 4 adjacent columns of
-// one chunk of 128 tokens and sums |X| sequentially in fp64 with 8-16 byte
-// loads (a warp reads 256-512 contiguous bytes per token row).  Phase 2: one
+// HBM-bound column reduction.  Phase 1: each thread owns 2 adjacent columns of
+// one chunk of 128 tokens and sums |X| sequentially in fp64, with 32 loads in
+// flight (a warp reads 128-256 contiguous bytes per token row).  Phase 2: one
 // thread per column adds the chunk partials in ascending chunk order, divides
 // by N in fp64 and rounds once to fp32.  The summation order is fixed, so the
 // result is bitwise reproducible.
@@ -24,40 +24,33 @@ __device__ __forceinline__ double abs_bf16_hi(uint32_t v) {
 template <bool BF16>
 __global__ void __launch_bounds__(128) stats_partial_kernel(const void *__restrict__ X, int64_t N,
                                                             int64_t I, double *__restrict__ part) {
-    const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // column quad
-    if (q * 4 >= I) return;
+    const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // column pair
+    if (q * 2 >= I) return;
     const int64_t c = blockIdx.y;
     const int64_t n0 = c * STATS_CHUNK;
     const int64_t n1 = (n0 + STATS_CHUNK < N) ? n0 + STATS_CHUNK : N;
-    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    double a0 = 0.0, a1 = 0.0;
+    const int64_t stride = I / 2;   // column pairs per row
     if constexpr (BF16) {
-        const int64_t stride = I / 4;  // uint2 per row
-        const uint2 *p = reinterpret_cast<const uint2 *>(X) + n0 * stride + q;
-#pragma unroll 16
+        const uint32_t *p = reinterpret_cast<const uint32_t *>(X) + n0 * stride + q;
+#pragma unroll 32
         for (int64_t n = n0; n < n1; ++n) {
-            const uint2 v = __ldg(p);
+            const uint32_t v = __ldg(p);
             p += stride;
-            a0 += abs_bf16_lo(v.x);
-            a1 += abs_bf16_hi(v.x);
-            a2 += abs_bf16_lo(v.y);
-            a3 += abs_bf16_hi(v.y);
+            a0 += abs_bf16_lo(v);
+            a1 += abs_bf16_hi(v);
         }
     } else {
-        const int64_t stride = I / 4;  // float4 per row
-        const float4 *p = reinterpret_cast<const float4 *>(X) + n0 * stride + q;
-#pragma unroll 8
+        const float2 *p = reinterpret_cast<const float2 *>(X) + n0 * stride + q;
+#pragma unroll 32
         for (int64_t n = n0; n < n1; ++n) {
-            const float4 v = __ldg(p);
+            const float2 v = __ldg(p);
             p += stride;
             a0 += fabs(static_cast<double>(v.x));
             a1 += fabs(static_cast<double>(v.y));
-            a2 += fabs(static_cast<double>(v.z));
-            a3 += fabs(static_cast<double>(v.w));
         }
     }
-    double2 *dst = reinterpret_cast<double2 *>(part + c * I + q * 4);
-    dst[0] = make_double2(a0, a1);
-    dst[1] = make_double2(a2, a3);
+    reinterpret_cast<double2 *>(part + c * I)[q] = make_double2(a0, a1);
 }
 
 __global__ void __launch_bounds__(256) stats_final_kernel(const double *__restrict__ part,
@@ -148,8 +141,8 @@ __global__ void __launch_bounds__(256) to_f16_kernel(const void *__restrict__ X,
 cudaError_t launch_stats_partial(const void *X, bool x_bf16, int64_t N, int64_t I, double *part,
                                  cudaStream_t st) {
     const int64_t n_chunks = (N + STATS_CHUNK - 1) / STATS_CHUNK;
-    const int64_t quads = I / 4;
-    dim3 grid(static_cast<unsigned>((quads + 127) / 128), static_cast<unsigned>(n_chunks));
+    const int64_t pairs = I / 2;
+    dim3 grid(static_cast<unsigned>((pairs + 127) / 128), static_cast<unsigned>(n_chunks));
     if (x_bf16)
         stats_partial_kernel<true><<<grid, 128, 0, st>>>(X, N, I, part);
     else
