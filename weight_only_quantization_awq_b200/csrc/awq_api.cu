@@ -452,9 +452,31 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     int sms;
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M <= 4) {
+        // decode: CUDA-core kernels streaming the packed weights
+        kt_reset(3);
+        kt_begin(3, st);
+        AWQ_CUDA(awq::launch_w4a16(x, M, in, out, qweight, scales, zeros, s16, group_size, y, st));
+        kt_end(3, st);
+        return AWQ_OK;
+    }
+    // prefill-sized M: tensor cores
+    const awq::TcPlan plan = awq::w4a16_tc_plan(M, in, out, sms);
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(plan.xs_bytes + plan.part_bytes + plan.counter_bytes)) return s;
+    char *wsp = ws.take<char>(plan.xs_bytes + plan.part_bytes + plan.counter_bytes);
+    awq::TcMaps maps;
+    if (awq_status_t s = make_map_2d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, qweight, in / 8, out,
+                                     8, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return s;
+    if (awq_status_t s = make_map_2d(&maps.xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, wsp, in, M,
+                                     awq::SLAB_K, static_cast<uint32_t>(plan.n_tile),
+                                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return s;
     kt_reset(3);
     kt_begin(3, st);
-    AWQ_CUDA(awq::launch_w4a16(x, M, in, out, qweight, scales, zeros, s16, group_size, y, st));
+    AWQ_CUDA(awq::launch_w4a16_tc(x, M, in, out, scales, zeros, s16, group_size, y, plan, wsp, maps,
+                                  st));
     kt_end(3, st);
     return AWQ_OK;
 }

@@ -229,8 +229,10 @@ __global__ void __launch_bounds__(512) w4a16_gemv_kernel(
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int e = wd * 8 + j + 4 * h;
-                    const float rs = __frcp_rn(__half2float(__ushort_as_half(sh[e])));
-                    v[h] = (active && m < M) ? __uint_as_float(static_cast<uint32_t>(xh[e]) << 16) * rs : 0.0f;
+                    v[h] = (active && m < M)
+                               ? __fdividef(__uint_as_float(static_cast<uint32_t>(xh[e]) << 16),
+                                            __half2float(__ushort_as_half(sh[e])))
+                               : 0.0f;
                     lsum[m] += v[h];
                 }
                 xr[m][wd * 4 + j] = make_float2(v[0] * inv16, v[1] * inv16);

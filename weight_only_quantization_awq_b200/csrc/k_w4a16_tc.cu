@@ -1,0 +1,410 @@
+// W4A16 linear on the tensor cores, for prefill-sized M (AWQ guide, section 三,
+// QuantLinear.forward: y = (x / s) * dequant(W)^T).
+//
+//   xs_absmax_kernel + xs_perm_kernel: xs = fp16((x / s16) * 2^-k), the power of
+//                   two chosen from max |x / s16| so the largest magnitude lands in
+//                   [2^14, 2^15), with the 8 columns of each packed word stored in
+//                   the order (0,4,1,5,2,6,3,7) (see below); y is scaled back by 2^k.
+//   w4a16_tc_kernel: one CTA per (128-row tile, token tile of <= 256, K split).
+//     warp 4 (TMA)  streams the packed codes [128 rows x 8 words] and the xs tile
+//                   [N tokens x 64 columns] of each 64-column slab into a ring;
+//     warps 0-3     dequantise: thread = row; a word's nibbles e and e+4 become one
+//                   fp16x2 (1024 + code) with a shift and a LOP3 against the 0x6400
+//                   magic; an exact HSUB2 of (1024 + z) and an HMUL2 by
+//                   Delta * 2^-kd (kd from max Delta, so the products stay normal
+//                   fp16) give the pair's dequantised weights with one rounding,
+//                   written to the 128B-swizzled K-major A tile.  The pair order
+//                   (e, e+4) is why xs is permuted the same way: the contraction
+//                   over K is order-independent.  y = accumulator * 2^(kx + kd).
+//     warp 5 (MMA)  one thread issues tcgen05.mma M=128 N=tokens K=16 (fp16 in,
+//                   fp32 accumulate in TMEM).
+//     warps 0-3     epilogue: tcgen05.ld of the accumulator; with one K split
+//                   y is written directly, otherwise each split stores fp32
+//                   partials and the last CTA of the tile (counter) adds them in
+//                   split order and writes y, so the result is deterministic.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "awq_internal.h"
+#include "awq_ptx.cuh"
+
+namespace awq {
+
+namespace {
+
+constexpr int TC_THREADS = 192;
+constexpr int TC_WARP_TMA = 4;
+constexpr int TC_WARP_MMA = 5;
+constexpr int TC_TOKENS = 256;       // max tokens per tile (MMA N)
+constexpr int RS = 4;                // input ring stages
+constexpr int AS_TC = 2;             // A ring stages
+constexpr int Q_BYTES = 128 * 32;    // packed codes of a slab: 128 rows x 8 words
+constexpr int A_BYTES = 128 * 128;   // bf16 A tile of a slab
+
+__device__ __forceinline__ int perm8(int p) { return (p >> 1) + 4 * (p & 1); }   // position -> column
+
+// max |x / s16| into max_bits[0] and max |Delta| into max_bits[2] (bit patterns of
+// non-negative floats order as their values).
+__global__ void __launch_bounds__(256) xs_absmax_kernel(const uint16_t *__restrict__ x,
+                                                        const uint16_t *__restrict__ s16, int64_t M,
+                                                        int64_t I, const uint16_t *__restrict__ scales,
+                                                        int64_t n_scales, unsigned *__restrict__ max_bits) {
+    float m = 0.0f, d = 0.0f;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < M * I; k += step) {
+        const int64_t c = k % I;
+        m = fmaxf(m, fabsf(__fdiv_rn(__uint_as_float(static_cast<uint32_t>(x[k]) << 16),
+                                     __half2float(__ushort_as_half(s16[c])))));
+    }
+    for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n_scales; k += step)
+        d = fmaxf(d, fabsf(__half2float(__ushort_as_half(scales[k]))));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        d = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, off));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicMax(max_bits, __float_as_uint(m));
+        atomicMax(max_bits + 2, __float_as_uint(d));
+    }
+}
+
+// Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero max).
+__device__ __forceinline__ int pow2_exp(float mx, int top) {
+    if (!(mx > 0.0f) || isinf(mx)) return 0;
+    int e;
+    frexpf(mx, &e);                                   // mx = f * 2^e, f in [0.5, 1)
+    const int k = e - top;
+    return k < -100 ? -100 : (k > 100 ? 100 : k);
+}
+
+// words: [0] max |xs| bits, [1] kx, [2] max |Delta| bits, [3] kd.
+__global__ void xs_perm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ s16,
+                               int64_t M, int64_t I, unsigned *__restrict__ words,
+                               uint16_t *__restrict__ xs) {
+    const int k = pow2_exp(__uint_as_float(words[0]), 15);       // max |xs| -> [2^14, 2^15)
+    const float sc = ldexpf(1.0f, -k);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        words[1] = static_cast<unsigned>(k);
+        words[3] = static_cast<unsigned>(pow2_exp(__uint_as_float(words[2]), 11));   // 15 * max Delta < 2^15
+    }
+    const int64_t total = M * I;
+    for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
+         q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t m = q / I, c = q % I;
+        const int64_t src = (c & ~int64_t(7)) + perm8(static_cast<int>(c & 7));
+        const float v = __fdiv_rn(__uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16),
+                                  __half2float(__ushort_as_half(s16[src])));
+        xs[q] = __half_as_ushort(__float2half_rn(v * sc));
+    }
+}
+
+struct TcArgs {
+    int64_t M, I, O;
+    int gs;
+    int n_tile;            // tokens per tile (multiple of 16, <= 256)
+    int splits;            // K splits
+    int slabs_per_split;
+    const uint16_t *scales;
+    const uint32_t *zeros;
+    uint16_t *y;
+    float *part;           // [splits][M][O] fp32 (splits > 1)
+    unsigned *counter;     // [row tiles * token tiles] (splits > 1), zeroed
+    const unsigned *words; // [1] kx, [3] kd: the accumulator is y * 2^-(kx + kd)
+};
+
+__device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
+    __half2 r = __hsub2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t h2mul(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+__device__ __forceinline__ uint32_t h2pack(float a) {
+    const __half2 h = __floats2half2_rn(a, a);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+template <bool ZEROS>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    w4a16_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int xs_bytes = a.n_tile * 128;
+    const int in_stage = (Q_BYTES + xs_bytes + 1023) / 1024 * 1024;
+    uint8_t *a_ring = base;                                  // AS_TC x 16 KB (1024-aligned)
+    uint8_t *in_ring = a_ring + AS_TC * A_BYTES;             // RS x (xs tile | codes)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(in_ring + RS * in_stage);
+    uint64_t *in_full = bars, *in_empty = bars + RS;
+    uint64_t *a_full = in_empty + RS, *a_empty = a_full + AS_TC;
+    uint64_t *acc_full = a_empty + AS_TC, *drain = acc_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *is_last = abort_flag + 1;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+    const int64_t OT = (a.O + 127) / 128;
+    const int64_t tile = blockIdx.x / a.splits;              // (token tile, row tile)
+    const int split = static_cast<int>(blockIdx.x % a.splits);
+    const int64_t ot = tile % OT, mt = tile / OT;
+    const int64_t nK = a.I / SLAB_K;
+    const int64_t kb0 = static_cast<int64_t>(split) * a.slabs_per_split;
+    const int64_t kb1 = kb0 + a.slabs_per_split < nK ? kb0 + a.slabs_per_split : nK;
+    const int nslab = static_cast<int>(kb1 > kb0 ? kb1 - kb0 : 0);
+    const uint32_t tcols = a.n_tile <= 32 ? 32 : (a.n_tile <= 64 ? 64 : (a.n_tile <= 128 ? 128 : 256));
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&in_full[s], 1);
+            mbar_init(&in_empty[s], 4 + 1);      // 4 dequant warps read the codes, the MMA reads xs
+        }
+        for (int s = 0; s < AS_TC; ++s) {
+            mbar_init(&a_full[s], 4);
+            mbar_init(&a_empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        *is_last = 0;
+        fence_mbar_init();
+    }
+    if (warp == TC_WARP_MMA) {
+        tmem_alloc(tmem_slot, tcols);
+        tmem_relinquish();
+    }
+    if (warp == TC_WARP_TMA && lane == 0) {
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.xs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == TC_WARP_TMA) {
+        if (lane == 0) {
+            int64_t last[RS];
+#pragma unroll
+            for (int s = 0; s < RS; ++s) last[s] = -1;
+            for (int i = 0; i < nslab; ++i) {
+                const uint32_t st = i % RS;
+                if (!mbar_wait(&in_empty[st], ((i / RS) & 1u) ^ 1u, abort_flag)) break;
+                uint8_t *dst = in_ring + st * in_stage;
+                const int32_t kb = static_cast<int32_t>(kb0 + i);
+                mbar_arrive_expect_tx(&in_full[st], Q_BYTES + xs_bytes);
+                tma_load_2d(dst, &maps.xs, &in_full[st], kb * SLAB_K, static_cast<int32_t>(mt * TC_TOKENS));
+                tma_load_2d(dst + xs_bytes, &maps.q, &in_full[st], kb * 8, static_cast<int32_t>(ot * 128));
+#pragma unroll
+                for (int s = 0; s < RS; ++s)
+                    if (s == static_cast<int>(st)) last[s] = i;
+            }
+#pragma unroll
+            for (int s = 0; s < RS; ++s)
+                if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / RS) & 1));
+        }
+        __syncwarp();
+    } else if (warp == TC_WARP_MMA) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16_f32(128, a.n_tile, false);
+            const uint32_t a_base = smem_u32(a_ring), in_base = smem_u32(in_ring);
+            bool ok = true;
+            for (int i = 0; i < nslab && ok; ++i) {
+                const uint32_t st = i % RS, as = i % AS_TC;
+                if (!mbar_wait(&a_full[as], (i / AS_TC) & 1u, abort_flag) ||
+                    !mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = a_base + as * A_BYTES;
+                const uint32_t b_addr = in_base + st * in_stage;
+#pragma unroll
+                for (int k = 0; k < SLAB_K / 16; ++k)
+                    umma_f16(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
+                             sdesc_kmajor_sw128(b_addr + k * 32), idesc, (i > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&in_empty[st]);
+                umma_commit(&a_empty[as]);
+            }
+            if (ok) umma_commit(acc_full);
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+        __syncwarp();
+    } else {
+        // ---- dequantisation: thread = row of the tile.
+        const int r = threadIdx.x;            // 0..127
+        const int64_t o = ot * 128 + r;
+        const bool row_ok = o < a.O;
+        const int64_t nG = a.I / a.gs, nzw = (nG + 7) / 8;
+        const float dscale = ldexpf(1.0f, -static_cast<int>(a.words[3]));
+        bool ok = true;
+        for (int i = 0; i < nslab; ++i) {
+            const uint32_t st = i % RS, as = i % AS_TC;
+            const int64_t kb = kb0 + i;
+            // group parameters of this row for the slab's one or two groups:
+            // Delta * 2^-kd and 1024 + z (both exact in fp16)
+            uint32_t dz[2][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t g = (kb * SLAB_K + h * 32) / a.gs;
+                float d = 0.0f, z = 8.0f;
+                if (row_ok) {
+                    d = __half2float(__ushort_as_half(__ldg(a.scales + o * nG + g)));
+                    if (ZEROS) z = static_cast<float>((__ldg(a.zeros + o * nzw + g / 8) >> (4 * (g % 8))) & 0xFu);
+                }
+                dz[h][0] = h2pack(d * dscale);
+                dz[h][1] = h2pack(1024.0f + z);
+            }
+            if (!mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&a_empty[as], ((i / AS_TC) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            const uint8_t *q = in_ring + st * in_stage + xs_bytes + r * 32;
+            const int c0 = (r >> 2) & 1;      // read order avoids bank conflicts between rows r and r+4
+            uint4 qw[2];
+            qw[c0] = *reinterpret_cast<const uint4 *>(q + 16 * c0);
+            qw[c0 ^ 1] = *reinterpret_cast<const uint4 *>(q + 16 * (c0 ^ 1));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&in_empty[st]);   // codes read (xs is released by the MMA)
+            uint8_t *dst = a_ring + as * A_BYTES;
+            const uint32_t wv[8] = {qw[0].x, qw[0].y, qw[0].z, qw[0].w, qw[1].x, qw[1].y, qw[1].z, qw[1].w};
+#pragma unroll
+            for (int wd = 0; wd < 8; ++wd) {
+                const int h = wd >> 2;
+                uint32_t v[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd
+                    const uint32_t b = ((wv[wd] >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
+                    v[e] = h2mul(h2sub(b, dz[h][1]), dz[h][0]);
+                }
+                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, wd)) = make_uint4(v[0], v[1], v[2], v[3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[as]);
+        }
+        // ---- epilogue
+        named_bar_sync(1, 128);
+        const bool got = ok && nslab > 0 && mbar_wait_sleep(acc_full, 0, abort_flag);
+        tc_fence_after();
+        const int64_t m0 = mt * TC_TOKENS;
+        const int mcount = static_cast<int>(a.M - m0 < a.n_tile ? a.M - m0 : a.n_tile);
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const float yscale = ldexpf(1.0f, static_cast<int>(a.words[1]) + static_cast<int>(a.words[3]));
+        if (__all_sync(0xffffffffu, got)) {
+            for (int c = 0; c < a.n_tile; c += 16) {
+                uint32_t rv[16];
+                tmem_ld16_wait(lane_addr + static_cast<uint32_t>(c), rv);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const int n = c + k;
+                    if (n < mcount && row_ok) {
+                        const float v = __uint_as_float(rv[k]) * yscale;
+                        if (a.splits == 1)
+                            a.y[(m0 + n) * a.O + o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                        else
+                            a.part[(static_cast<int64_t>(split) * a.M + m0 + n) * a.O + o] = v;
+                    }
+                }
+            }
+        }
+        if (a.splits > 1) {
+            __threadfence();
+            named_bar_sync(1, 128);
+            if (threadIdx.x == 0) {
+                const unsigned prev = atomicAdd(&a.counter[tile], 1u);
+                *is_last = prev == static_cast<unsigned>(a.splits - 1);
+            }
+            named_bar_sync(1, 128);
+            if (*is_last) {
+                __threadfence();
+                if (row_ok) {
+                    for (int n = 0; n < mcount; ++n) {
+                        float t = 0.0f;
+                        for (int s = 0; s < a.splits; ++s)
+                            t += __ldcg(a.part + (static_cast<int64_t>(s) * a.M + m0 + n) * a.O + o);
+                        a.y[(m0 + n) * a.O + o] = __bfloat16_as_ushort(__float2bfloat16_rn(t));
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == TC_WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, tcols);
+    }
+}
+
+}  // namespace
+
+TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
+    TcPlan p;
+    const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
+    const int64_t nK = I / SLAB_K;
+    int64_t splits = (2 * num_sms + OT * MT - 1) / (OT * MT);
+    if (splits < 1) splits = 1;
+    if (splits > nK) splits = nK;
+    const int64_t spl = (nK + splits - 1) / splits;
+    splits = (nK + spl - 1) / spl;
+    p.splits = static_cast<int>(splits);
+    p.slabs_per_split = static_cast<int>(spl);
+    p.n_tile = static_cast<int>(M >= TC_TOKENS ? TC_TOKENS : (M + 15) / 16 * 16);
+    p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
+    p.part_bytes = splits > 1 ? (splits * M * O * 4 + 255) / 256 * 256 : 0;
+    p.counter_bytes = (OT * MT * 4 + 16 + 255) / 256 * 256;   // 4 scale words, tile counters
+    return p;
+}
+
+cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
+                            const uint16_t *scales, const uint32_t *zeros, const uint16_t *s16,
+                            int gs, uint16_t *y, const TcPlan &plan, char *workspace,
+                            const TcMaps &maps, cudaStream_t st) {
+    const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(workspace);
+    float *part = plan.splits > 1 ? reinterpret_cast<float *>(workspace + plan.xs_bytes) : nullptr;
+    unsigned *words = reinterpret_cast<unsigned *>(workspace + plan.xs_bytes + plan.part_bytes);
+    unsigned *xw = words;                                       // [4]: max|xs|, kx, max|Delta|, kd
+    unsigned *counter = words + 4;                              // [OT * MT]
+    cudaError_t e = cudaMemsetAsync(words, 0, plan.counter_bytes, st);
+    if (e != cudaSuccess) return e;
+    int blocks = static_cast<int>((M * I + 255) / 256);
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    xs_absmax_kernel<<<blocks, 256, 0, st>>>(x, s16, M, I, scales, O * (I / gs), xw);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    xs_perm_kernel<<<blocks, 256, 0, st>>>(x, s16, M, I, xw, xs);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    TcArgs a;
+    a.M = M;
+    a.I = I;
+    a.O = O;
+    a.gs = gs;
+    a.n_tile = plan.n_tile;
+    a.splits = plan.splits;
+    a.slabs_per_split = plan.slabs_per_split;
+    a.scales = scales;
+    a.zeros = zeros;
+    a.y = y;
+    a.part = part;
+    a.counter = counter;
+    a.words = xw;
+    const int in_stage = (Q_BYTES + plan.n_tile * 128 + 1023) / 1024 * 1024;
+    const int smem = 1024 + AS_TC * A_BYTES + RS * in_stage + (2 * RS + 2 * AS_TC + 2) * 8 + 16;
+    const unsigned grid = static_cast<unsigned>(OT * MT * plan.splits);
+    if (zeros) {
+        e = cudaFuncSetAttribute(w4a16_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        w4a16_tc_kernel<true><<<grid, TC_THREADS, smem, st>>>(maps, a);
+    } else {
+        e = cudaFuncSetAttribute(w4a16_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        w4a16_tc_kernel<false><<<grid, TC_THREADS, smem, st>>>(maps, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace awq
