@@ -265,6 +265,8 @@ def run_ours(args, rank, world, local_rank):
     apply_bytes = O * I // 2 + O * (I // GROUP) * 2 + I * 2 + APPLY_M * I * 2 + APPLY_M * O * 2
     del g
 
+    block_apply = measure_block_apply(dev)
+
     pk_ = peaks()
     search_kernel_ms = statistics.mean(search_ms) if search_ms else None
     achieved = flops_step / (search_kernel_ms * 1e-3) / 1e12 if search_kernel_ms else None
@@ -305,11 +307,72 @@ def run_ours(args, rank, world, local_rank):
                   "gb_per_s": round(apply_bytes / (apply_us * 1e-6) / 1e9, 1),
                   "frac_hbm": round(apply_bytes / (apply_us * 1e-6) / 1e9 / pk_["hbm_gbs"], 4),
                   "bytes": apply_bytes, "timing": f"CUDA graph of {reps * n_copies} launches over {n_copies} packed copies"},
+        "w4a16_block": {str(m): {**v, "frac_hbm": round(v["gb_per_s"] / pk_["hbm_gbs"], 4)}
+                        for m, v in block_apply.items()},
     }
     if rank == 0 and world == 1:
         out["cpu_baseline"] = cpu_baseline(W_np, X_np)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
+    return out
+
+
+def measure_block_apply(dev, ms=(1, 16, 256), copies=2, reps=4):
+    """W4A16 apply over the seven linears of the Llama-7B decoder block (q, k, v, o
+    4096x4096; gate, up 11008x4096; down 4096x11008), asymmetric INT4 g128, for
+    each M: one CUDA graph replays `reps` passes over `copies` packed copies of
+    the block (2 x 105 MB > L2).  Weights are seeded bf16 draws packed on the GPU."""
+    import torch
+    import weight_only_quantization_awq_b200 as awq
+    from synthetic import BLOCK_LINEARS
+    gen = torch.Generator(device=dev).manual_seed(20261202)
+    packs = []
+    for c in range(copies):
+        layer = []
+        for name, o, i in BLOCK_LINEARS:
+            W = (torch.randn((o, i), generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+            sX = torch.rand(i, generator=gen, device=dev) + 0.5
+            layer.append((awq.awq_pack_int4(W, sX, 0.5, 1.0, GROUP, "asym"), o, i))
+            del W
+        packs.append(layer)
+    torch.cuda.synchronize()
+    out = {}
+    for m in ms:
+        xs = {i: (torch.randn((m, i), generator=gen, device=dev)).to(torch.bfloat16)
+              for i in {i for _, _, i in BLOCK_LINEARS}}
+        ys = [torch.empty((m, o), dtype=torch.bfloat16, device=dev) for _, o, _ in BLOCK_LINEARS]
+
+        def run_block(layer):
+            for k, (p, o, i) in enumerate(layer):
+                awq.awq_linear_w4a16(xs[i], p["qweight"], p["scales"], p["zeros"], p["s16"], GROUP,
+                                     out=ys[k])
+
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for layer in packs:
+                run_block(layer)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                for layer in packs:
+                    run_block(layer)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+        byts = sum(p["qweight"].numel() * 4 + p["scales"].numel() * 2 + p["zeros"].numel() * 4 +
+                   p["s16"].numel() * 2 + m * i * 2 + m * o * 2 for p, o, i in packs[0])
+        flops = sum(2.0 * m * o * i for _, o, i in BLOCK_LINEARS)
+        out[m] = {"us_per_block": round(us, 2), "gb_per_s": round(byts / (us * 1e-6) / 1e9, 1),
+                  "tflops": round(flops / (us * 1e-6) / 1e12, 2), "bytes": byts}
+        del g
     return out
 
 

@@ -135,7 +135,7 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in,
  * per group, linear):
  *     y[m, o] = sum_i (x[m, i] / s16[i]) * (code[o, i] - z[o, i/gs]) * scales[o, i/gs]
  * with z = 8 when zeros == NULL (symmetric storage).  fp32 accumulation.
- * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.
+ * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.  in <= 49152.
  * Storage arguments as produced by awq_pack_int4.  Asynchronous.
  */
 awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,

@@ -94,7 +94,8 @@ struct TcPlan {
     int64_t xs_bytes, part_bytes, counter_bytes;   // workspace pieces (256-byte rounded)
 };
 TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms);
-// workspace: xs (plan.xs_bytes) then part (plan.part_bytes) then counters and two words.
+// workspace: xs (plan.xs_bytes), the fp32 split-K accumulator (plan.part_bytes), then
+// four scale words and the tile counters (plan.counter_bytes).
 cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const uint16_t *scales, const uint32_t *zeros, const uint16_t *s16,
                             int gs, uint16_t *y, const TcPlan &plan, char *workspace,

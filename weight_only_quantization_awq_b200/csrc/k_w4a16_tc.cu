@@ -6,9 +6,10 @@
 //                   [2^14, 2^15), with the 8 columns of each packed word stored in
 //                   the order (0,4,1,5,2,6,3,7) (see below); y is scaled back by 2^k.
 //   w4a16_tc_kernel: one CTA per (128-row tile, token tile of <= 256, K split).
-//     warp 4 (TMA)  streams the packed codes [128 rows x 8 words] and the xs tile
+//     warp 8 (TMA)  streams the packed codes [128 rows x 8 words] and the xs tile
 //                   [N tokens x 64 columns] of each 64-column slab into a ring;
-//     warps 0-3     dequantise: thread = row; a word's nibbles e and e+4 become one
+//     warps 0-7     dequantise: two threads per row (32 columns each); the next
+//                   slab's Delta and z are loaded one slab ahead; a word's nibbles e and e+4 become one
 //                   fp16x2 (1024 + code) with a shift and a LOP3 against the 0x6400
 //                   magic; an exact HSUB2 of (1024 + z) and an HMUL2 by
 //                   Delta * 2^-kd (kd from max Delta, so the products stay normal
@@ -16,12 +17,13 @@
 //                   written to the 128B-swizzled K-major A tile.  The pair order
 //                   (e, e+4) is why xs is permuted the same way: the contraction
 //                   over K is order-independent.  y = accumulator * 2^(kx + kd).
-//     warp 5 (MMA)  one thread issues tcgen05.mma M=128 N=tokens K=16 (fp16 in,
+//     warp 9 (MMA)  one thread issues tcgen05.mma M=128 N=tokens K=16 (fp16 in,
 //                   fp32 accumulate in TMEM).
 //     warps 0-3     epilogue: tcgen05.ld of the accumulator; with one K split
-//                   y is written directly, otherwise each split stores fp32
-//                   partials and the last CTA of the tile (counter) adds them in
-//                   split order and writes y, so the result is deterministic.
+//                   y is written directly, otherwise each split adds its fp32
+//                   partial into a zeroed fp32 tile with red.global.add (the order
+//                   of those adds across splits is not fixed) and the last CTA of
+//                   the tile (counter) converts the tile to bf16.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -32,12 +34,13 @@ namespace awq {
 
 namespace {
 
-constexpr int TC_THREADS = 192;
-constexpr int TC_WARP_TMA = 4;
-constexpr int TC_WARP_MMA = 5;
+constexpr int TC_DQ_WARPS = 8;       // dequantisation warps (2 threads per row)
+constexpr int TC_WARP_TMA = 8;
+constexpr int TC_WARP_MMA = 9;
+constexpr int TC_THREADS = 10 * 32;
 constexpr int TC_TOKENS = 256;       // max tokens per tile (MMA N)
 constexpr int RS = 4;                // input ring stages
-constexpr int AS_TC = 2;             // A ring stages
+constexpr int AS_MAX = 8;            // A ring stages: as many as shared memory allows, up to 8
 constexpr int Q_BYTES = 128 * 32;    // packed codes of a slab: 128 rows x 8 words
 constexpr int A_BYTES = 128 * 128;   // bf16 A tile of a slab
 
@@ -53,8 +56,8 @@ __global__ void __launch_bounds__(256) xs_absmax_kernel(const uint16_t *__restri
     const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < M * I; k += step) {
         const int64_t c = k % I;
-        m = fmaxf(m, fabsf(__fdiv_rn(__uint_as_float(static_cast<uint32_t>(x[k]) << 16),
-                                     __half2float(__ushort_as_half(s16[c])))));
+        m = fmaxf(m, fabsf(__fdividef(__uint_as_float(static_cast<uint32_t>(x[k]) << 16),
+                                      __half2float(__ushort_as_half(s16[c])))));
     }
     for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n_scales; k += step)
         d = fmaxf(d, fabsf(__half2float(__ushort_as_half(scales[k]))));
@@ -93,8 +96,8 @@ __global__ void xs_perm_kernel(const uint16_t *__restrict__ x, const uint16_t *_
          q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t m = q / I, c = q % I;
         const int64_t src = (c & ~int64_t(7)) + perm8(static_cast<int>(c & 7));
-        const float v = __fdiv_rn(__uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16),
-                                  __half2float(__ushort_as_half(s16[src])));
+        const float v = __fdividef(__uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16),
+                                   __half2float(__ushort_as_half(s16[src])));
         xs[q] = __half_as_ushort(__float2half_rn(v * sc));
     }
 }
@@ -105,10 +108,11 @@ struct TcArgs {
     int n_tile;            // tokens per tile (multiple of 16, <= 256)
     int splits;            // K splits
     int slabs_per_split;
+    int as;                // A ring stages
     const uint16_t *scales;
     const uint32_t *zeros;
     uint16_t *y;
-    float *part;           // [splits][M][O] fp32 (splits > 1)
+    float *acc32;          // [M][O] fp32, zeroed (splits > 1)
     unsigned *counter;     // [row tiles * token tiles] (splits > 1), zeroed
     const unsigned *words; // [1] kx, [3] kd: the accumulator is y * 2^-(kx + kd)
 };
@@ -134,12 +138,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int xs_bytes = a.n_tile * 128;
     const int in_stage = (Q_BYTES + xs_bytes + 1023) / 1024 * 1024;
-    uint8_t *a_ring = base;                                  // AS_TC x 16 KB (1024-aligned)
-    uint8_t *in_ring = a_ring + AS_TC * A_BYTES;             // RS x (xs tile | codes)
+    const int AS = a.as;
+    uint8_t *a_ring = base;                                  // AS x 16 KB (1024-aligned)
+    uint8_t *in_ring = a_ring + AS * A_BYTES;                // RS x (xs tile | codes)
     uint64_t *bars = reinterpret_cast<uint64_t *>(in_ring + RS * in_stage);
     uint64_t *in_full = bars, *in_empty = bars + RS;
-    uint64_t *a_full = in_empty + RS, *a_empty = a_full + AS_TC;
-    uint64_t *acc_full = a_empty + AS_TC, *drain = acc_full + 1;
+    uint64_t *a_full = in_empty + RS, *a_empty = a_full + AS_MAX;
+    uint64_t *acc_full = a_empty + AS_MAX, *drain = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *is_last = abort_flag + 1;
@@ -158,10 +163,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < RS; ++s) {
             mbar_init(&in_full[s], 1);
-            mbar_init(&in_empty[s], 4 + 1);      // 4 dequant warps read the codes, the MMA reads xs
+            mbar_init(&in_empty[s], TC_DQ_WARPS + 1);   // dequant warps read the codes, the MMA reads xs
         }
-        for (int s = 0; s < AS_TC; ++s) {
-            mbar_init(&a_full[s], 4);
+        for (int s = 0; s < AS; ++s) {
+            mbar_init(&a_full[s], TC_DQ_WARPS);
             mbar_init(&a_empty[s], 1);
         }
         mbar_init(acc_full, 1);
@@ -211,8 +216,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint32_t a_base = smem_u32(a_ring), in_base = smem_u32(in_ring);
             bool ok = true;
             for (int i = 0; i < nslab && ok; ++i) {
-                const uint32_t st = i % RS, as = i % AS_TC;
-                if (!mbar_wait(&a_full[as], (i / AS_TC) & 1u, abort_flag) ||
+                const uint32_t st = i % RS, as = i % AS;
+                if (!mbar_wait(&a_full[as], (i / AS) & 1u, abort_flag) ||
                     !mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -233,58 +238,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---- dequantisation: thread = row of the tile.
-        const int r = threadIdx.x;            // 0..127
+        // ---- dequantisation: two threads per row, 32 columns (4 packed words) each.
+        const int r = threadIdx.x >> 1, hh = threadIdx.x & 1;
         const int64_t o = ot * 128 + r;
         const bool row_ok = o < a.O;
         const int64_t nG = a.I / a.gs, nzw = (nG + 7) / 8;
         const float dscale = ldexpf(1.0f, -static_cast<int>(a.words[3]));
+        // Delta and (1024 + z) of this thread's group in slab i (fp16x2, exact).
+        auto group_params = [&](int i, uint32_t &d2, uint32_t &z2) {
+            float d = 0.0f, z = 8.0f;
+            if (row_ok && i < nslab) {
+                const int64_t g = ((kb0 + i) * SLAB_K + hh * 32) / a.gs;
+                d = __half2float(__ushort_as_half(__ldg(a.scales + o * nG + g)));
+                if (ZEROS) z = static_cast<float>((__ldg(a.zeros + o * nzw + g / 8) >> (4 * (g % 8))) & 0xFu);
+            }
+            d2 = h2pack(d * dscale);
+            z2 = h2pack(1024.0f + z);
+        };
+        uint32_t d_cur, z_cur, d_nxt, z_nxt;
+        group_params(0, d_cur, z_cur);
         bool ok = true;
         for (int i = 0; i < nslab; ++i) {
-            const uint32_t st = i % RS, as = i % AS_TC;
-            const int64_t kb = kb0 + i;
-            // group parameters of this row for the slab's one or two groups:
-            // Delta * 2^-kd and 1024 + z (both exact in fp16)
-            uint32_t dz[2][2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int64_t g = (kb * SLAB_K + h * 32) / a.gs;
-                float d = 0.0f, z = 8.0f;
-                if (row_ok) {
-                    d = __half2float(__ushort_as_half(__ldg(a.scales + o * nG + g)));
-                    if (ZEROS) z = static_cast<float>((__ldg(a.zeros + o * nzw + g / 8) >> (4 * (g % 8))) & 0xFu);
-                }
-                dz[h][0] = h2pack(d * dscale);
-                dz[h][1] = h2pack(1024.0f + z);
-            }
+            const uint32_t st = i % RS, as = i % AS;
+            group_params(i + 1, d_nxt, z_nxt);            // one slab ahead
             if (!mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) { ok = false; break; }
-            if (!mbar_wait(&a_empty[as], ((i / AS_TC) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-            const uint8_t *q = in_ring + st * in_stage + xs_bytes + r * 32;
-            const int c0 = (r >> 2) & 1;      // read order avoids bank conflicts between rows r and r+4
-            uint4 qw[2];
-            qw[c0] = *reinterpret_cast<const uint4 *>(q + 16 * c0);
-            qw[c0 ^ 1] = *reinterpret_cast<const uint4 *>(q + 16 * (c0 ^ 1));
+            if (!mbar_wait(&a_empty[as], ((i / AS) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+            const uint4 qw = *reinterpret_cast<const uint4 *>(in_ring + st * in_stage + xs_bytes + r * 32 + hh * 16);
             __syncwarp();
             if (lane == 0) mbar_arrive(&in_empty[st]);   // codes read (xs is released by the MMA)
             uint8_t *dst = a_ring + as * A_BYTES;
-            const uint32_t wv[8] = {qw[0].x, qw[0].y, qw[0].z, qw[0].w, qw[1].x, qw[1].y, qw[1].z, qw[1].w};
+            const uint32_t wv[4] = {qw.x, qw.y, qw.z, qw.w};
 #pragma unroll
-            for (int wd = 0; wd < 8; ++wd) {
-                const int h = wd >> 2;
+            for (int wd = 0; wd < 4; ++wd) {
                 uint32_t v[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd
                     const uint32_t b = ((wv[wd] >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
-                    v[e] = h2mul(h2sub(b, dz[h][1]), dz[h][0]);
+                    v[e] = h2mul(h2sub(b, z_cur), d_cur);
                 }
-                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, wd)) = make_uint4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, hh * 4 + wd)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[as]);
+            d_cur = d_nxt;
+            z_cur = z_nxt;
         }
-        // ---- epilogue
+        if (warp < 4) {
+        // ---- epilogue (warps 0-3): thread = TMEM lane = row of the tile
+        const int64_t eo = ot * 128 + threadIdx.x;
+        const bool erow_ok = eo < a.O;
         named_bar_sync(1, 128);
         const bool got = ok && nslab > 0 && mbar_wait_sleep(acc_full, 0, abort_flag);
         tc_fence_after();
@@ -299,12 +303,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     const int n = c + k;
-                    if (n < mcount && row_ok) {
+                    if (n < mcount && erow_ok) {
                         const float v = __uint_as_float(rv[k]) * yscale;
                         if (a.splits == 1)
-                            a.y[(m0 + n) * a.O + o] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                            a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
                         else
-                            a.part[(static_cast<int64_t>(split) * a.M + m0 + n) * a.O + o] = v;
+                            atomicAdd(a.acc32 + (m0 + n) * a.O + eo, v);   // result unused: red.global.add
                     }
                 }
             }
@@ -319,15 +323,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             named_bar_sync(1, 128);
             if (*is_last) {
                 __threadfence();
-                if (row_ok) {
-                    for (int n = 0; n < mcount; ++n) {
-                        float t = 0.0f;
-                        for (int s = 0; s < a.splits; ++s)
-                            t += __ldcg(a.part + (static_cast<int64_t>(s) * a.M + m0 + n) * a.O + o);
-                        a.y[(m0 + n) * a.O + o] = __bfloat16_as_ushort(__float2bfloat16_rn(t));
-                    }
+                if (erow_ok) {
+#pragma unroll 8
+                    for (int n = 0; n < mcount; ++n)
+                        a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(
+                            __float2bfloat16_rn(__ldcg(a.acc32 + (m0 + n) * a.O + eo)));
                 }
             }
+        }
         }
     }
     tc_fence_before();
@@ -344,7 +347,10 @@ TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     TcPlan p;
     const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
     const int64_t nK = I / SLAB_K;
-    int64_t splits = (2 * num_sms + OT * MT - 1) / (OT * MT);
+    // wide token tiles: about one CTA per SM (the split-K adds grow with the splits);
+    // narrow ones: about two per SM, for latency hiding
+    const int64_t target = M >= 128 ? num_sms : 2 * num_sms;
+    int64_t splits = target / (OT * MT);          // at most one wave
     if (splits < 1) splits = 1;
     if (splits > nK) splits = nK;
     const int64_t spl = (nK + splits - 1) / splits;
@@ -353,7 +359,7 @@ TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     p.slabs_per_split = static_cast<int>(spl);
     p.n_tile = static_cast<int>(M >= TC_TOKENS ? TC_TOKENS : (M + 15) / 16 * 16);
     p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
-    p.part_bytes = splits > 1 ? (splits * M * O * 4 + 255) / 256 * 256 : 0;
+    p.part_bytes = splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
     p.counter_bytes = (OT * MT * 4 + 16 + 255) / 256 * 256;   // 4 scale words, tile counters
     return p;
 }
@@ -364,11 +370,12 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const TcMaps &maps, cudaStream_t st) {
     const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
     uint16_t *xs = reinterpret_cast<uint16_t *>(workspace);
-    float *part = plan.splits > 1 ? reinterpret_cast<float *>(workspace + plan.xs_bytes) : nullptr;
+    float *acc32 = plan.splits > 1 ? reinterpret_cast<float *>(workspace + plan.xs_bytes) : nullptr;
     unsigned *words = reinterpret_cast<unsigned *>(workspace + plan.xs_bytes + plan.part_bytes);
     unsigned *xw = words;                                       // [4]: max|xs|, kx, max|Delta|, kd
     unsigned *counter = words + 4;                              // [OT * MT]
-    cudaError_t e = cudaMemsetAsync(words, 0, plan.counter_bytes, st);
+    // one memset zeroes the fp32 accumulator tile (if any), the scale words and the counters
+    cudaError_t e = cudaMemsetAsync(workspace + plan.xs_bytes, 0, plan.part_bytes + plan.counter_bytes, st);
     if (e != cudaSuccess) return e;
     int blocks = static_cast<int>((M * I + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
@@ -389,11 +396,18 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     a.scales = scales;
     a.zeros = zeros;
     a.y = y;
-    a.part = part;
+    a.acc32 = acc32;
     a.counter = counter;
     a.words = xw;
     const int in_stage = (Q_BYTES + plan.n_tile * 128 + 1023) / 1024 * 1024;
-    const int smem = 1024 + AS_TC * A_BYTES + RS * in_stage + (2 * RS + 2 * AS_TC + 2) * 8 + 16;
+    const int fixed = 1024 + RS * in_stage + (2 * RS + 2 * AS_MAX + 2) * 8 + 16;
+    // Deep enough that dequantisation runs well ahead of the MMA completions, but
+    // keep two CTAs per SM when the token tile is narrow.
+    int as = (113 * 1024 - fixed) / A_BYTES;
+    if (as < 3) as = (227 * 1024 - fixed) / A_BYTES;
+    as = as > AS_MAX ? AS_MAX : (as < 2 ? 2 : as);
+    a.as = as;
+    const int smem = fixed + as * A_BYTES;
     const unsigned grid = static_cast<unsigned>(OT * MT * plan.splits);
     if (zeros) {
         e = cudaFuncSetAttribute(w4a16_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
