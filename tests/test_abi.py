@@ -54,6 +54,7 @@ def _search(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(W=NULL), ARG), (dict(wdt=7), ARG), (dict(out=0), ARG), (dict(quant=2), ARG),
     (dict(gs=96), UNSUP), (dict(gs=256), UNSUP), (dict(inp=520), UNSUP), (dict(wbit=3), UNSUP),
+    (dict(inp=576), UNSUP),          # a multiple of 64 that 128-column groups do not divide
     (dict(W=FAKE + 8), ALIGN), (dict(X=FAKE + 4), ALIGN), (dict(na=0), ARG), (dict(na=65), ARG),
     (dict(nc=-1), ARG), (dict(clip=NULL), ARG), (dict(N=0), ARG), (dict(loss=NULL), ARG),
     (dict(alpha=(ctypes.c_double * 20)(*([0.5] * 19 + [1.5]))), ARG),
@@ -88,6 +89,7 @@ def test_pack_rejects_on_host():
     assert call({5: ctypes.c_double(-0.1)}) == ARG
     assert call({6: ctypes.c_double(0.0)}) == ARG
     assert call({7: 48}) == UNSUP
+    assert call({3: 320}) == UNSUP               # in = 320 is not a whole number of 128-column groups
     assert call({9: FAKE + 4}) == ALIGN
     assert call({4: NULL}) == ARG
 
@@ -103,5 +105,6 @@ def test_linear_rejects_on_host():
     assert call({0: NULL}) == ARG
     assert call({1: 0}) == ARG
     assert call({2: 100}) == UNSUP
+    assert call({2: 4160}) == UNSUP              # multiple of 64, not of the 128-column group
     assert call({8: 16}) == UNSUP
     assert call({0: FAKE + 2}) == ALIGN

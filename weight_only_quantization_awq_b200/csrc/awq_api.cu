@@ -208,6 +208,8 @@ awq_status_t check_layer(const void *W, int w_dtype, int64_t out, int64_t in, in
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
     if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 64", (long long)in);
+    if (in % group_size != 0)
+        return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of group_size %d", (long long)in, group_size);
     if (in > (1 << 20) || out > (1 << 24)) return fail(AWQ_ERR_UNSUPPORTED, "layer too large");
     if (!aligned16(W)) return fail(AWQ_ERR_ALIGN, "W not 16-byte aligned");
     return AWQ_OK;
@@ -444,6 +446,8 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
     if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 64", (long long)in);
+    if (in % group_size != 0)
+        return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of group_size %d", (long long)in, group_size);
     if (in > 49152) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld above 49152", (long long)in);
     if (!aligned16(x) || !aligned16(qweight) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
         (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)) || !aligned16(s16) ||

@@ -102,6 +102,11 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const TcMaps &maps, cudaStream_t st);
 
 // ---- W4A16 apply
+// Streaming GEMV for 1 <= M <= 4 (activations staged per CTA; see k_w4a16_stream.cu).
+bool w4a16_stream_supported(int64_t M, int64_t I);
+cudaError_t launch_w4a16_stream(const uint16_t *x, int64_t M, int64_t I, int64_t O,
+                                const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
+                                const uint16_t *s16, int gs, uint16_t *y, int num_sms, cudaStream_t st);
 cudaError_t launch_w4a16(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                          const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
                          const uint16_t *s16, int gs, uint16_t *y, cudaStream_t st);

@@ -101,7 +101,39 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Wait until the preceding kernel of the stream has completed and its memory is
+// visible (returns at once when the launch has no programmatic dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next kernel of the stream (launched with programmatic stream
+// serialisation) to start its pre-wait part.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Hint: bring [p, p + bytes) into L2 (bulk, asynchronous, no completion).  The
+// range is shrunk to 16-byte boundaries, so nothing outside it is touched.
+__device__ __forceinline__ void l2_prefetch_range(const void *p, uint64_t bytes) {
+    uint64_t a = (reinterpret_cast<uint64_t>(p) + 15) & ~uint64_t(15);
+    const uint64_t e = (reinterpret_cast<uint64_t>(p) + bytes) & ~uint64_t(15);
+    while (a < e) {
+        const uint32_t n = static_cast<uint32_t>(e - a < 32768 ? e - a : 32768);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(n) : "memory");
+        a += n;
+    }
+}
+
 // ----------------------------------------------------------------------- TMA
+// Plain (untiled) bulk copy global -> this CTA's shared memory, completion
+// signalled on `bar` as transaction bytes.  Both addresses 16-byte aligned,
+// bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -4,7 +4,8 @@
 //     y[m, o] = sum_g Delta[o, g] * ( sum_{i in g} xs[m, i] * code[o, i]  -  z[o, g] * sum_{i in g} xs[m, i] )
 //     xs = x / s16
 //
-// Decode kernel for small M, bound by HBM at M = 1.  One warp streams one
+// Fallback decode kernel for M <= 4 at input widths whose activations the
+// streaming kernel (k_w4a16_stream.cu) cannot stage.  One warp streams one
 // output row at a time: each lane owns 4 consecutive packed words (32 columns,
 // inside one group) of every 1024-column block of the row and issues all of
 // its 16-byte loads before using any.  A nibble becomes an exact float with a
@@ -156,157 +157,6 @@ __global__ void __launch_bounds__(W4_THREADS) w4a16_decode_kernel(
     }
 }
 
-// ---------------------------------------------------------------------------
-// Split-K GEMV for M <= 2.  A block has one warp per 1024-column block of the
-// row (NB warps, NB <= 16).  Each warp keeps the activations of its lane's 32
-// columns in registers for the whole kernel (pre-divided by s and by 16^j), so
-// its row loop is only 16-byte loads, LOP3, FADD2 and FFMA2: about 2 ALU ops per
-// weight.  The warps' per-row partial sums meet in shared memory, 8 rows at a
-// time, and one warp writes y.
-constexpr int GV_ROWS = 8;
-
-template <int MT, bool ZEROS>
-__global__ void __launch_bounds__(512) w4a16_gemv_kernel(
-    const uint16_t *__restrict__ x, int M, int I, int64_t O,
-    const uint32_t *__restrict__ qweight, const uint16_t *__restrict__ scales,
-    const uint32_t *__restrict__ zeros, const uint16_t *__restrict__ s16, int gs,
-    uint16_t *__restrict__ y, int64_t rows_per_block) {
-    __shared__ float red[GV_ROWS][MT][33];
-    const int NB = blockDim.x / 32;
-    const int b = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = b * BLK_COLS + lane * 32;        // this lane's 32 columns
-    const bool active = c < I;
-    const int nG = I / gs;
-    const int64_t nzw = (nG + 7) / 8;
-    const int g = active ? c / gs : 0;
-
-    const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per_block;
-    const int64_t r1 = r0 + rows_per_block < O ? r0 + rows_per_block : O;
-    uint4 qv[GV_ROWS];
-    float dv[GV_ROWS], zv[GV_ROWS];
-    auto load_chunk = [&](int64_t o0) {
-#pragma unroll
-        for (int r = 0; r < GV_ROWS; ++r) {
-            const int64_t o = o0 + r;
-            qv[r] = make_uint4(0u, 0u, 0u, 0u);
-            dv[r] = 0.0f;
-            zv[r] = 0.0f;
-            if (active && o < r1) {
-                qv[r] = __ldg(reinterpret_cast<const uint4 *>(qweight + o * (I / 8) + c / 8));
-                dv[r] = __half2float(__ushort_as_half(__ldg(scales + o * nG + g)));
-                zv[r] = ZEROS ? static_cast<float>((__ldg(zeros + o * nzw + g / 8) >> (4 * (g % 8))) & 0xFu)
-                              : 8.0f;
-            }
-        }
-    };
-    // The first chunk's weights are requested before anything else, so their
-    // latency overlaps the activation set-up below.
-    load_chunk(r0);
-
-    // Activations of this lane's columns: pair (wd, j) = columns (8wd + j, 8wd + j + 4),
-    // divided by s and by 16^j; lsum = their plain sum (for the zero point).
-    float2 xr[MT][16];
-    float lsum[MT];
-#pragma unroll
-    for (int m = 0; m < MT; ++m) {
-        lsum[m] = 0.0f;
-        uint4 xv[4] = {}, sv[4] = {};
-        if (active && m < M) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                xv[q] = __ldg(reinterpret_cast<const uint4 *>(x + static_cast<int64_t>(m) * I + c) + q);
-                sv[q] = __ldg(reinterpret_cast<const uint4 *>(s16 + c) + q);
-            }
-        }
-        const uint16_t *xh = reinterpret_cast<const uint16_t *>(xv);
-        const uint16_t *sh = reinterpret_cast<const uint16_t *>(sv);
-#pragma unroll
-        for (int wd = 0; wd < 4; ++wd) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float inv16 = j == 0 ? 1.0f : (j == 1 ? 0.0625f : (j == 2 ? 0.00390625f : 0.000244140625f));
-                float v[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int e = wd * 8 + j + 4 * h;
-                    v[h] = (active && m < M)
-                               ? __fdividef(__uint_as_float(static_cast<uint32_t>(xh[e]) << 16),
-                                            __half2float(__ushort_as_half(sh[e])))
-                               : 0.0f;
-                    lsum[m] += v[h];
-                }
-                xr[m][wd * 4 + j] = make_float2(v[0] * inv16, v[1] * inv16);
-            }
-        }
-    }
-
-    const float2 NEGM = make_float2(-MAGIC23, -MAGIC23);
-    for (int64_t o0 = r0; o0 < r1; o0 += GV_ROWS) {
-        if (o0 != r0) load_chunk(o0);
-#pragma unroll
-        for (int r = 0; r < GV_ROWS; ++r) {
-            float2 part[MT];
-#pragma unroll
-            for (int m = 0; m < MT; ++m) part[m] = make_float2(0.0f, 0.0f);
-            const uint32_t wds[4] = {qv[r].x, qv[r].y, qv[r].z, qv[r].w};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-                const uint32_t lo = wds[wd], hi = wds[wd] >> 16;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint32_t mask = 0xFu << (4 * j);
-                    const float2 f = make_float2(__uint_as_float((lo & mask) | 0x4B000000u),
-                                                 __uint_as_float((hi & mask) | 0x4B000000u));
-                    const float2 q = __fadd2_rn(f, NEGM);               // code * 16^j, exact
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) part[m] = __ffma2_rn(q, xr[m][wd * 4 + j], part[m]);
-                }
-            }
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                float v = dv[r] * (part[m].x + part[m].y - zv[r] * lsum[m]);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) red[r][m][b] = v;
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x < GV_ROWS * MT) {
-            const int r = threadIdx.x / MT, m = threadIdx.x % MT;
-            const int64_t o = o0 + r;
-            if (o < r1 && m < M) {
-                float t = 0.0f;
-                for (int k = 0; k < NB; ++k) t += red[r][m][k];
-                y[static_cast<int64_t>(m) * O + o] = __bfloat16_as_ushort(__float2bfloat16_rn(t));
-            }
-        }
-        __syncthreads();
-    }
-}
-
-template <int MT, bool ZEROS>
-cudaError_t launch_gemv(const uint16_t *x, int64_t M, int64_t I, int64_t O,
-                        const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
-                        const uint16_t *s16, int gs, uint16_t *y, cudaStream_t st) {
-    const int NB = static_cast<int>((I + BLK_COLS - 1) / BLK_COLS);
-    int dev = 0, sms = 148, per_sm = 1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, w4a16_gemv_kernel<MT, ZEROS>,
-                                                      NB * 32, 0);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-    // One wave; rows split evenly in multiples of GV_ROWS.
-    int64_t blocks = static_cast<int64_t>(sms) * per_sm;
-    int64_t rpb = (O + blocks - 1) / blocks;
-    rpb = (rpb + GV_ROWS - 1) / GV_ROWS * GV_ROWS;
-    blocks = (O + rpb - 1) / rpb;
-    w4a16_gemv_kernel<MT, ZEROS><<<static_cast<unsigned>(blocks), NB * 32, 0, st>>>(
-        x, static_cast<int>(M), static_cast<int>(I), O, qweight, scales, zeros, s16, gs, y, rpb);
-    return cudaGetLastError();
-}
-
 template <int MT, bool ZEROS>
 cudaError_t launch_decode(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                           const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
@@ -348,12 +198,13 @@ cudaError_t launch_w4a16(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     // Tokens per pass: as many as fit the block's staged activations (<= 227 KB).
     const int64_t per_token = 4 * (((I + BLK_COLS - 1) / BLK_COLS) * (BLK_COLS + 32));
     const bool z = zeros != nullptr;
-    if (M <= 2 && I <= 16 * BLK_COLS) {
-        if (M == 1)
-            return z ? launch_gemv<1, true>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st)
-                     : launch_gemv<1, false>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st);
-        return z ? launch_gemv<2, true>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st)
-                 : launch_gemv<2, false>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st);
+    if (M <= 4 && w4a16_stream_supported(M, I)) {
+        int dev = 0, sms = 148;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        return launch_w4a16_stream(x, M, I, O, qweight, scales, zeros, s16, gs, y, sms, st);
     }
 #define AWQ_DEC(MT)                                                                      \
     return z ? launch_decode<MT, true>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st) \
