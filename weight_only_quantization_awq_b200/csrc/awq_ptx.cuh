@@ -124,16 +124,6 @@ __device__ __forceinline__ void l2_prefetch_range(const void *p, uint64_t bytes)
 }
 
 // ----------------------------------------------------------------------- TMA
-// Plain (untiled) bulk copy global -> this CTA's shared memory, completion
-// signalled on `bar` as transaction bytes.  Both addresses 16-byte aligned,
-// bytes a multiple of 16.
-__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
