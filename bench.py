@@ -43,7 +43,11 @@ APPLY_M = 1
 # DRAM traffic of one search-kernel launch on this workload, from the ncu capture
 # summarised in profiles/search_kernel_attn_proj_4096x4096_n4096.md, valid only for the
 # kernel source it was taken on (sha256 of csrc/k_search.cu, first 16 hex).
-SEARCH_TRAFFIC = {"source_sha": "f07af1a0ea671b9c", "bytes": 353965568}
+# Kernels of one step: statistics 2 (partial, final); search 9 (absmax, fp16 copy,
+# scale table 2, group parameters, search, row and block reductions, argmin);
+# packing 3 (scale table 2, pack); apply 1.
+LAUNCHES_PER_STEP = 15
+SEARCH_TRAFFIC = {"source_sha": "c1c00c0da8de7e66", "bytes": 346585600}
 
 
 def _env_int(k, d):
@@ -291,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"},
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 13 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
         "roofline": {"bound": "tensor", "kernel": "search_kernel",
                      "achieved": round(achieved, 2) if achieved else None,
