@@ -124,6 +124,24 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- our arm
+def max_over_ranks(value, world, device=None):
+    """The largest `value` over all ranks (a job takes as long as its slowest
+    rank); `value` itself when there is one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step, steps, world, ms):
+    """Whole-job throughput: each of `world` ranks runs `steps` steps of its own
+    layer, all within `ms` milliseconds (the max over ranks)."""
+    return flops_per_step * steps * world / (ms * 1e-3) / 1e12
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -186,13 +204,9 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms / args.steps
-    value = flops_step * args.steps * world / (ms * 1e-3) / 1e12
+    value = job_tflops(flops_step, args.steps, world, ms)
 
     # ---- end to end through the public API: pinned host inputs in, results out.
     W_h = torch.from_numpy(W_np.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -229,14 +243,10 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = W_h.numel() * 2 + X_h.numel() * 2 + x_h.numel() * 2
     d2h = qh.numel() * 4 + sh.numel() * 2 + s16h.numel() * 2 + yh.numel() * 2 + 8 * G + 4 * 8
-    e2e_value = flops_step * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = job_tflops(flops_step, e2e_steps, world, e2e_ms)
 
     # ---- W4A16 apply at M = 1: rotating packed copies (> L2), one CUDA graph of launches.
     n_copies = 16
