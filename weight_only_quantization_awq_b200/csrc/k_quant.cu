@@ -112,7 +112,15 @@ __global__ void __launch_bounds__(128) group_params_kernel(
         wr[4 * k] = v.x; wr[4 * k + 1] = v.y; wr[4 * k + 2] = v.z; wr[4 * k + 3] = v.w;
     }
     for (int g = 0; g < G; ++g) {
-        float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
+        // four independent max / min chains (max and min are exact, so the split
+        // changes no result), merged at the end
+        float mx4[4], mn4[4], am4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            mx4[k] = -3.4028234663852886e38f;
+            mn4[k] = 3.4028234663852886e38f;
+            am4[k] = 0.0f;
+        }
 #pragma unroll
         for (int e4 = 0; e4 < GS / 4; ++e4) {
             const float4 s4 = *reinterpret_cast<const float4 *>(&s_sm[g][4 * e4]);
@@ -127,13 +135,16 @@ __global__ void __launch_bounds__(128) group_params_kernel(
                     w = __uint_as_float(wr[e]);
                 const float wp = __fmul_rn(w, sv[k]);
                 if (asym) {
-                    mx = fmaxf(mx, wp);
-                    mn = fminf(mn, wp);
+                    mx4[k] = fmaxf(mx4[k], wp);
+                    mn4[k] = fminf(mn4[k], wp);
                 } else {
-                    amax = fmaxf(amax, fabsf(wp));
+                    am4[k] = fmaxf(am4[k], fabsf(wp));
                 }
             }
         }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+        const float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
+        const float amax = fmaxf(fmaxf(am4[0], am4[1]), fmaxf(am4[2], am4[3]));
         const double r = clip.value[g];
         float D, qlo, qhi;
         if (!asym) {
@@ -174,132 +185,172 @@ cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I
 }
 
 // -------------------------------------------------------------------- pack
-// One thread per packed word (8 consecutive columns of a row).  The gs/8
-// threads of a group are consecutive lanes of one warp and reduce with xor
-// shuffles; the first of them writes the group's scale and zero point.
+// 2-D grid: blockIdx.x = row, a thread packs PW consecutive words (8 columns
+// each) of that row, issuing all of its loads (W and s) before any arithmetic.
+// A group's gs/8 words belong to gs/(8*PW) consecutive lanes (or to part of
+// one thread's words), which reduce with xor shuffles; the group's first
+// thread writes its scale and zero point.
+constexpr int PACK_PW = 4;                   // words per thread
+constexpr int PACK_THREADS = 128;
+
 template <bool WBF16>
-__global__ void __launch_bounds__(256) pack_kernel(const void *__restrict__ W, int64_t O, int64_t I,
-                                                   int gs, bool asym, double clip,
-                                                   const float *__restrict__ s,
-                                                   uint32_t *__restrict__ qweight,
-                                                   uint16_t *__restrict__ scales,
-                                                   uint32_t *__restrict__ zeros,
-                                                   uint16_t *__restrict__ s16,
-                                                   float *__restrict__ scales_f32) {
-    const int64_t wpr = I / 8;
-    const int64_t total = O * wpr;
-    const int seg = gs / 8;
-    const int64_t nG = I / gs;
-    const int64_t nzw = (nG + 7) / 8;
-    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const int64_t iters = (total + step - 1) / step;
-    for (int64_t it = 0; it < iters; ++it) {
-        const int64_t idx = it * step + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-        const bool active = idx < total;
-        const int64_t o = active ? idx / wpr : 0;
-        const int64_t wcol = active ? idx % wpr : 0;
-        const int64_t c0 = wcol * 8;
-        float w[8], sv[8], wp[8];
-        if (active) {
-            if constexpr (WBF16) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(W) +
-                                                                o * I + c0);
-                const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+__global__ void __launch_bounds__(PACK_THREADS) pack_kernel(const void *__restrict__ W, int O, int I,
+                                                            int gs, bool asym, double clip,
+                                                            const float *__restrict__ s,
+                                                            uint32_t *__restrict__ qweight,
+                                                            uint16_t *__restrict__ scales,
+                                                            uint32_t *__restrict__ zeros,
+                                                            uint16_t *__restrict__ s16,
+                                                            float *__restrict__ scales_f32) {
+    const int o = blockIdx.x;
+    const int wpr = I / 8;                                  // words per row
+    const int w0 = (blockIdx.y * PACK_THREADS + threadIdx.x) * PACK_PW;   // first word of this thread
+    const int nG = I / gs, nzw = (nG + 7) / 8;
+    const int wpg = gs / 8;                                 // words per group (4, 8 or 16)
+    const bool active = w0 < wpr;                           // wpr is a multiple of PACK_PW (I % 64 == 0)
+    // ---- loads: W (PW x 8 values) and s (PW x 8 values)
+    float w[PACK_PW][8], sv[PACK_PW][8];
+    if (active) {
+        if constexpr (WBF16) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(W) +
+                                                               static_cast<int64_t>(o) * I) + w0;
+            uint4 v[PACK_PW];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    w[2 * k] = __uint_as_float(u[k] << 16);
-                    w[2 * k + 1] = __uint_as_float(u[k] & 0xFFFF0000u);
+            for (int k = 0; k < PACK_PW; ++k) v[k] = __ldg(src + k);
+#pragma unroll
+            for (int k = 0; k < PACK_PW; ++k) {
+                const uint32_t u[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    w[k][2 * e] = __uint_as_float(u[e] << 16);
+                    w[k][2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
                 }
-            } else {
-                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(W) +
-                                                                  o * I + c0);
-                const float4 a = p[0], b = p[1];
-                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-                w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
             }
-            const float4 sa = *reinterpret_cast<const float4 *>(s + c0);
-            const float4 sb = *reinterpret_cast<const float4 *>(s + c0 + 4);
-            sv[0] = sa.x; sv[1] = sa.y; sv[2] = sa.z; sv[3] = sa.w;
-            sv[4] = sb.x; sv[5] = sb.y; sv[6] = sb.z; sv[7] = sb.w;
         } else {
+            const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(W) +
+                                                                 static_cast<int64_t>(o) * I) + 2 * w0;
+            float4 v[2 * PACK_PW];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) { w[k] = 0.0f; sv[k] = 1.0f; }
-        }
-        float mx = -3.4028234663852886e38f, mn = 3.4028234663852886e38f, amax = 0.0f;
+            for (int k = 0; k < 2 * PACK_PW; ++k) v[k] = __ldg(src + k);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            wp[k] = __fmul_rn(w[k], sv[k]);
-            mx = fmaxf(mx, wp[k]);
-            mn = fminf(mn, wp[k]);
-            amax = fmaxf(amax, fabsf(wp[k]));
+            for (int k = 0; k < PACK_PW; ++k) {
+                w[k][0] = v[2 * k].x; w[k][1] = v[2 * k].y; w[k][2] = v[2 * k].z; w[k][3] = v[2 * k].w;
+                w[k][4] = v[2 * k + 1].x; w[k][5] = v[2 * k + 1].y; w[k][6] = v[2 * k + 1].z; w[k][7] = v[2 * k + 1].w;
+            }
         }
-        for (int off = 1; off < seg; off <<= 1) {
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float4 *sp = reinterpret_cast<const float4 *>(s) + 2 * w0;
+        float4 sq[2 * PACK_PW];
+#pragma unroll
+        for (int k = 0; k < 2 * PACK_PW; ++k) sq[k] = __ldg(sp + k);
+#pragma unroll
+        for (int k = 0; k < PACK_PW; ++k) {
+            sv[k][0] = sq[2 * k].x; sv[k][1] = sq[2 * k].y; sv[k][2] = sq[2 * k].z; sv[k][3] = sq[2 * k].w;
+            sv[k][4] = sq[2 * k + 1].x; sv[k][5] = sq[2 * k + 1].y; sv[k][6] = sq[2 * k + 1].z; sv[k][7] = sq[2 * k + 1].w;
         }
-        float D, z = 0.0f;
-        if (!asym) {
-            const float a = clip == 1.0 ? amax : __double2float_rn(__dmul_rn((double)amax, clip));
-            D = __fdiv_rn(a, 7.0f);
-        } else {
-            const float hi = clip == 1.0 ? mx : __double2float_rn(__dmul_rn((double)mx, clip));
-            const float lo = clip == 1.0 ? mn : __double2float_rn(__dmul_rn((double)mn, clip));
-            D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
-            if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+    } else {
+#pragma unroll
+        for (int k = 0; k < PACK_PW; ++k)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) { w[k][e] = 0.0f; sv[k][e] = 1.0f; }
+    }
+    // ---- per word: W' = W * s and its group bounds
+    float wp[PACK_PW][8], mx[PACK_PW], mn[PACK_PW], am[PACK_PW];
+#pragma unroll
+    for (int k = 0; k < PACK_PW; ++k) {
+        mx[k] = -3.4028234663852886e38f;
+        mn[k] = 3.4028234663852886e38f;
+        am[k] = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            wp[k][e] = __fmul_rn(w[k][e], sv[k][e]);
+            mx[k] = fmaxf(mx[k], wp[k][e]);
+            mn[k] = fminf(mn[k], wp[k][e]);
+            am[k] = fmaxf(am[k], fabsf(wp[k][e]));
         }
-        // q = rint(RN(W'/Delta)) from the reciprocal product W' * RN(1/Delta): every
-        // decision that survives the clamp has |W'/Delta| <= 15.5, where the product
-        // is within 2^-19 of RN(W'/Delta); products within 2^-16 of a half-integer
-        // (exact ties included) are redone with the correctly rounded division.
+    }
+    // words of one thread that share a group (gs = 32: 4 words per group, the thread's
+    // PW = 4 words are exactly one group; larger groups span 2 or 4 lanes)
+    float gmx = mx[0], gmn = mn[0], gam = am[0];
+#pragma unroll
+    for (int k = 1; k < PACK_PW; ++k) {
+        gmx = fmaxf(gmx, mx[k]);
+        gmn = fminf(gmn, mn[k]);
+        gam = fmaxf(gam, am[k]);
+    }
+    const int lpg = wpg / PACK_PW;                          // lanes per group: 1, 2 or 4
+    for (int off = 1; off < lpg; off <<= 1) {
+        gmx = fmaxf(gmx, __shfl_xor_sync(0xffffffffu, gmx, off));
+        gmn = fminf(gmn, __shfl_xor_sync(0xffffffffu, gmn, off));
+        gam = fmaxf(gam, __shfl_xor_sync(0xffffffffu, gam, off));
+    }
+    float D, z = 0.0f;
+    if (!asym) {
+        const float a = clip == 1.0 ? gam : __double2float_rn(__dmul_rn((double)gam, clip));
+        D = __fdiv_rn(a, 7.0f);
+    } else {
+        const float hi = clip == 1.0 ? gmx : __double2float_rn(__dmul_rn((double)gmx, clip));
+        const float lo = clip == 1.0 ? gmn : __double2float_rn(__dmul_rn((double)gmn, clip));
+        D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+        if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+    }
+    // q = rint(RN(W'/Delta)) from the reciprocal product W' * RN(1/Delta): every
+    // decision that survives the clamp has |W'/Delta| <= 15.5, where the product
+    // is within 2^-19 of RN(W'/Delta); products within 2^-16 of a half-integer
+    // (exact ties included) are redone with the correctly rounded division.
+    const float invD = D != 0.0f ? __frcp_rn(D) : 0.0f;
+    uint32_t word[PACK_PW];
+#pragma unroll
+    for (int k = 0; k < PACK_PW; ++k) {
         float q[8];
-        const float invD = D != 0.0f ? __frcp_rn(D) : 0.0f;
         bool near_tie = false;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            q[k] = __fsub_rn(__fmaf_rn(wp[k], invD, 12582912.0f), 12582912.0f);
-            near_tie |= fabsf(__fmaf_rn(wp[k], invD, -q[k])) > 0.5f - 1.0f / 65536.0f;
+        for (int e = 0; e < 8; ++e) {
+            q[e] = __fsub_rn(__fmaf_rn(wp[k][e], invD, 12582912.0f), 12582912.0f);
+            near_tie |= fabsf(__fmaf_rn(wp[k][e], invD, -q[e])) > 0.5f - 1.0f / 65536.0f;
         }
         if (near_tie && D != 0.0f) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) q[k] = rintf(__fdiv_rn(wp[k], D));
+            for (int e = 0; e < 8; ++e) q[e] = rintf(__fdiv_rn(wp[k][e], D));
         }
-        uint32_t word = 0;
+        uint32_t wd = 0;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float c = asym ? fminf(fmaxf(q[k] + z, 0.0f), 15.0f)
-                                 : fminf(fmaxf(q[k], -8.0f), 7.0f) + 8.0f;
-            word |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * k);
+        for (int e = 0; e < 8; ++e) {
+            const float c = asym ? fminf(fmaxf(q[e] + z, 0.0f), 15.0f) : fminf(fmaxf(q[e], -8.0f), 7.0f) + 8.0f;
+            wd |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * e);
         }
-        if (!active) continue;
-        qweight[idx] = word;
-        if ((wcol % seg) == 0) {
-            const int64_t j = c0 / gs;
-            scales[o * nG + j] = __half_as_ushort(__float2half_rn(D));
-            if (scales_f32) scales_f32[o * nG + j] = D;
-            if (zeros)
-                atomicOr(&zeros[o * nzw + j / 8],
-                         (static_cast<uint32_t>(z) & 0xFu) << (4 * static_cast<int>(j % 8)));
-        }
-        if (o == 0) {
+        word[k] = wd;
+    }
+    if (!active) return;
+    *reinterpret_cast<uint4 *>(qweight + static_cast<int64_t>(o) * wpr + w0) =
+        make_uint4(word[0], word[1], word[2], word[3]);
+    if ((w0 % wpg) == 0) {                                  // the group's first thread
+        const int j = w0 / wpg;
+        scales[static_cast<int64_t>(o) * nG + j] = __half_as_ushort(__float2half_rn(D));
+        if (scales_f32) scales_f32[static_cast<int64_t>(o) * nG + j] = D;
+        if (zeros)
+            atomicOr(&zeros[static_cast<int64_t>(o) * nzw + j / 8],
+                     (static_cast<uint32_t>(z) & 0xFu) << (4 * (j % 8)));
+    }
+    if (o == 0) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) s16[c0 + k] = __half_as_ushort(__float2half_rn(sv[k]));
-        }
+        for (int k = 0; k < PACK_PW; ++k)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s16[(w0 + k) * 8 + e] = __half_as_ushort(__float2half_rn(sv[k][e]));
     }
 }
 
 cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs, bool asym,
                         double clip, const float *s, uint32_t *qweight, uint16_t *scales,
                         uint32_t *zeros, uint16_t *s16, float *scales_f32, cudaStream_t st) {
-    const int64_t total = O * (I / 8);
-    int64_t blocks = (total + 255) / 256;
-    if (blocks > 148 * 8) blocks = 148 * 8;
+    const int64_t wpr = I / 8;
+    const dim3 grid(static_cast<unsigned>(O),
+                    static_cast<unsigned>((wpr / PACK_PW + PACK_THREADS - 1) / PACK_THREADS));
     if (w_bf16)
-        pack_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-            W, O, I, gs, asym, clip, s, qweight, scales, zeros, s16, scales_f32);
+        pack_kernel<true><<<grid, PACK_THREADS, 0, st>>>(W, static_cast<int>(O), static_cast<int>(I), gs, asym,
+                                                         clip, s, qweight, scales, zeros, s16, scales_f32);
     else
-        pack_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-            W, O, I, gs, asym, clip, s, qweight, scales, zeros, s16, scales_f32);
+        pack_kernel<false><<<grid, PACK_THREADS, 0, st>>>(W, static_cast<int>(O), static_cast<int>(I), gs, asym,
+                                                          clip, s, qweight, scales, zeros, s16, scales_f32);
     return cudaGetLastError();
 }
 
