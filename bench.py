@@ -212,16 +212,33 @@ def run_ours(args, rank, world, local_rank):
     W_h = torch.from_numpy(W_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     X_h = torch.from_numpy(X_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
-    Wd_e, Xd_e, xd_e = torch.empty_like(Ws[0]), torch.empty_like(Xs[0]), torch.empty_like(xd)
     qh = torch.empty(p["qweight"].shape, dtype=torch.int32).pin_memory()
     sh = torch.empty(p["scales"].shape, dtype=torch.float16).pin_memory()
     s16h = torch.empty(p["s16"].shape, dtype=torch.float16).pin_memory()
     yh = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
+    # Two device input buffers: step k+1's host-to-device copies run on a copy
+    # stream while step k computes (a layer-by-layer quantiser loads the next
+    # layer during the current one).  Every step still copies its own inputs.
+    comp_st = torch.cuda.current_stream()
+    copy_st = torch.cuda.Stream()
+    bufs = [(torch.empty_like(Ws[0]), torch.empty_like(Xs[0]), torch.empty_like(xd)) for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        Wd_e.copy_(W_h, non_blocking=True)
-        Xd_e.copy_(X_h, non_blocking=True)
-        xd_e.copy_(x_h, non_blocking=True)
+    def issue_copy(k):
+        b = k % 2
+        with torch.cuda.stream(copy_st):
+            if k >= 2:
+                copy_st.wait_event(done[b])          # step k-2 has finished with buffer b
+            bufs[b][0].copy_(W_h, non_blocking=True)
+            bufs[b][1].copy_(X_h, non_blocking=True)
+            bufs[b][2].copy_(x_h, non_blocking=True)
+            copied[b].record(copy_st)
+
+    def e2e_step(k):
+        b = k % 2
+        comp_st.wait_event(copied[b])
+        Wd_e, Xd_e, xd_e = bufs[b]
         sX = awq.awq_act_stats(Xd_e)
         r = awq.awq_search_layer(Wd_e, Xd_e, sX, GROUP, 4, "sym", alphas)
         pk = awq.awq_pack_int4(Wd_e, sX, alphas[r["best_alpha"]], 1.0, GROUP, "sym")
@@ -230,17 +247,25 @@ def run_ours(args, rank, world, local_rank):
         sh.copy_(pk["scales"], non_blocking=True)
         s16h.copy_(pk["s16"], non_blocking=True)
         yh.copy_(yy, non_blocking=True)
+        done[b].record(comp_st)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    def e2e_run(n, start=None):
+        if start is not None:
+            copy_st.wait_event(start)                # no copy begins before the timed region
+        issue_copy(0)
+        for k in range(n):
+            if k + 1 < n:
+                issue_copy(k + 1)
+            e2e_step(k)
+
+    e2e_run(max(2, args.warmup))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
     e2e_steps = max(1, min(args.steps, 50))
-    for _ in range(e2e_steps):
-        e2e_step()
+    e0.record()
+    e2e_run(e2e_steps, e0)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
@@ -297,7 +322,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": wl.name, "out": O, "in": I, "tokens": N, "grid": G,
                    "quant": "sym_int4", "group_size": GROUP, "apply_m": APPLY_M,
