@@ -137,6 +137,14 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in,
  * with z = 8 when zeros == NULL (symmetric storage).  fp32 accumulation.
  * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.  in <= 49152.
  * Storage arguments as produced by awq_pack_int4.  Asynchronous.
+ * Precision: x / s16 is rounded to fp16 after a power-of-two scale (2^-11
+ * relative); for M >= 5 (tensor cores) (code - z) * scale is also rounded to
+ * fp16 once.  M <= 4 runs on the CUDA cores and needs no workspace.
+ * Ordering: the M <= 4 kernel is launched with programmatic stream
+ * serialisation, so its blocks may start while the preceding kernel on
+ * `stream` is still running; until that kernel has completed they only ask L2
+ * to prefetch qweight, scales and zeros (a hint that reads nothing into the
+ * SM), and every read of an argument, and the write of y, happens after it.
  */
 awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
                               const uint32_t *qweight, const uint16_t *scales,
