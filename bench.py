@@ -124,6 +124,17 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- our arm
+def bench_config(wl, world):
+    """The workload description both arms report (one layer per rank)."""
+    from synthetic import ALPHA_GRID
+    L = wl.layers[0]
+    O, I, N = L.out, L.inp, wl.tokens
+    return {"workload": wl.name, "out": O, "in": I, "tokens": N, "grid": len(ALPHA_GRID),
+            "quant": "sym_int4", "group_size": GROUP, "apply_m": APPLY_M,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"}
+
+
 def max_over_ranks(value, world, device=None):
     """The largest `value` over all ranks (a job takes as long as its slowest
     rank); `value` itself when there is one rank."""
@@ -324,10 +335,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "out": O, "in": I, "tokens": N, "grid": G,
-                   "quant": "sym_int4", "group_size": GROUP, "apply_m": APPLY_M,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"},
+        "config": bench_config(wl, world),
         "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
@@ -474,8 +482,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": wl.name, "out": L.out, "in": L.inp, "tokens": wl.tokens,
-                       "grid": 20, "quant": "sym_int4", "group_size": GROUP},
+            "config": bench_config(wl, 1),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
