@@ -239,3 +239,36 @@ def test_linear_w4a16_block_shape(awq, M):
     y_ref = oracle.linear_w4a16(x, u32(p["qweight"]), u16(p["scales"]), u32(p["zeros"]),
                                 u16(p["s16"]), 128)
     check_apply(y, y_ref)
+
+
+@pytest.mark.parametrize("M", [1, 2, 4, 5])
+@pytest.mark.parametrize("pattern", ["tiny", "mixed", "zero"])
+def test_linear_w4a16_activation_range(awq, M, pattern):
+    """Activations far below 1 (whole rows near the bottom of the normal float
+    range), rows mixing tiny, zero and ordinary 32-column chunks, and all-zero
+    activations: every pass scales x / s by a power of two before rounding it to
+    fp16, and that scale must stay finite.  in = 1088 leaves a ragged last block
+    of 32-column chunks."""
+    O, I, gs = 96, 1088, 64
+    W, X = small_layer(O, I, 64, seed=M + 11)
+    p = oracle.pack_int4(W, oracle.act_stats(X), 0.5, 1.0, gs, 1)
+    xf = synthetic.bf16_to_f32(apply_activations(M, I, seed=M + 3)).astype(np.float64)
+    if pattern == "tiny":
+        xf *= 2.0 ** -118
+    elif pattern == "mixed":
+        xf[:, :256] *= 2.0 ** -118
+        xf[:, 256:512] = 0.0
+        xf[:, 1024:] *= 2.0 ** -60
+    else:
+        xf[:] = 0.0
+    x = synthetic.bf16_bits(xf.astype(np.float32))
+    y_ref = oracle.linear_w4a16(x, p["qweight"], p["scales"], p["zeros"], p["s16"], gs)
+    got = awq.awq_linear_w4a16(
+        dev(x), dev(p["qweight"].view(np.int32)), dev(p["scales"].view(np.float16)),
+        dev(p["zeros"].view(np.int32)), dev(p["s16"].view(np.float16)), gs)
+    y = got.float().cpu().numpy()
+    assert np.all(np.isfinite(y))
+    if pattern == "zero":
+        assert np.all(y == 0.0)
+    else:
+        check_apply(got, y_ref)

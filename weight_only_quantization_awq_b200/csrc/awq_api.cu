@@ -128,7 +128,8 @@ awq_status_t make_map_2d(CUtensorMap *map, CUtensorMapDataType dt, size_t elem, 
 
 // The search kernel's four tensor maps (out-of-bounds boxes read as zero, so
 // ragged rows and token tails contribute nothing):
-//   x  : fp16 copy of X [N, I], boxes of 64 channels x 256 tokens, 128B swizzle;
+//   x  : fp16 copy of X [N, I], boxes of 64 channels x 128 tokens (one CTA's half of
+//        a 256-token MMA tile), 128B swizzle;
 //   w  : W [O, I], 128 rows x 128 bytes per box, 128B swizzle;
 //   sn : scale table [2G, I] fp32, boxes of 64 channels x (s row, -1/s row);
 //   qp : group parameters [G * I/gs][O][4] fp32 (3-D), boxes of 128 rows x the
@@ -137,7 +138,7 @@ awq_status_t make_search_maps(awq::SearchMaps *m, const uint16_t *x16, int64_t N
                               bool w_bf16, int64_t O, int64_t I, const float *sn,
                               const float4 *qparam, int G, int gs) {
     if (awq_status_t s = make_map_2d(&m->x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x16, I, N,
-                                     awq::SLAB_K, awq::SUB_N, CU_TENSOR_MAP_SWIZZLE_128B))
+                                     awq::SLAB_K, awq::SUB_N / 2, CU_TENSOR_MAP_SWIZZLE_128B))
         return s;
     if (awq_status_t s = w_bf16 ? make_map_2d(&m->w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, I, O,
                                               64, awq::TILE_O, CU_TENSOR_MAP_SWIZZLE_128B)

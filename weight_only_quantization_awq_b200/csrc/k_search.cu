@@ -1,6 +1,6 @@
 // Fused AWQ grid-search kernel for sm_100a.
 //
-// For grid point g, output rows [128*ot, 128*ot + 128) and tokens
+// For grid point g, output rows [256*ot, 256*ot + 256) and tokens
 // [512*tb, 512*tb + 512), it accumulates
 //     E[o, n] = sum_i dW_g[o, i] * X[n, i],   dW_g = Q(W * s_g) / s_g - W
 // on the 5th-generation tensor cores (fp16 operands, fp32 accumulation) and
@@ -10,24 +10,35 @@
 // arithmetic), evaluated for every s = s_X^alpha on the grid.  Neither dW nor E
 // ever reaches global memory.
 //
-// Warp roles (704 threads, one CTA per SM, persistent over work units):
+// CTA pairs (clusters of two, one CTA per SM, persistent over work units) run
+// the pair form of the 5th-generation MMA: M = 256 rows, of which each CTA
+// forms and holds 128 (its own rows of dW), and N = 256 tokens per
+// instruction, of which each CTA stages 128 (half of each X tile).  Each CTA's
+// TMEM receives its 128 rows x all 512 tokens of the unit.  So each SM streams
+// half of the X tiles a single-CTA MMA of the same shape would need: X re-reads
+// from L2 are what bound the single-CTA form of this kernel.
+//
+// Warp roles (704 threads per CTA):
 //   warps 0-15  dW producers (16 columns of one row per thread): read one slab's
 //               inputs (W tile, s and -1/s, group parameters) from shared
-//               memory, form dW for 128 rows x 64 columns, write it as fp16 into
-//               shared memory in the 128-byte-swizzled K-major layout the MMA
-//               reads, signal a_full.
-//   warps 16-19 epilogue: tcgen05.ld of the 128 x 512 fp32 accumulator (lane =
-//               output row), square-and-sum per row, one fp32 partial per
-//               (grid point, token block, row).
-//   warp 20     TMA: lane 0 streams X tiles (256 tokens x 64 channels, fp16
-//               copy of X scaled by a power of two) into the X ring; lane 1
-//               streams each slab's producer inputs into the input ring.
-//   warp 21     MMA: allocates 512 TMEM columns; one thread issues
-//               tcgen05.mma M=128 N=256 K=16 (two N=256 halves per slab) and
-//               tcgen05.commit releases ring stages and the accumulator.
-// Work units are (g fastest, then output tile, then token block) and are dealt
-// round-robin to the CTAs, so the CTAs running at one time share a few W tiles
-// and X blocks in L2.
+//               memory, form dW for the CTA's 128 rows x 64 columns, write it
+//               as fp16 into shared memory in the 128-byte-swizzled K-major
+//               layout the MMA reads, arrive on the leader's a_full.
+//   warps 16-19 epilogue: tcgen05.ld of the CTA's 128 x 512 fp32 accumulator
+//               (lane = output row), square-and-sum per row, one fp32 partial
+//               per (grid point, token block, row).
+//   warp 20     TMA: lane 0 streams this CTA's half of the X tiles (128 tokens x
+//               64 channels, fp16 copy of X scaled by a power of two) into the X
+//               ring, counted on the leader's x_full; lane 1 streams each slab's
+//               producer inputs into the (local) input ring.
+//   warp 21     MMA: both CTAs allocate 512 TMEM columns as a pair; in the
+//               leader (rank 0) one thread issues tcgen05.mma.cta_group::2
+//               M=256 N=256 K=16 (two N=256 halves per slab), and
+//               tcgen05.commit with a multicast arrive releases both CTAs' ring
+//               stages and accumulators.
+// Work units are (g fastest, then 256-row output tile, then token block) and
+// are dealt round-robin to the pairs, so the pairs running at one time share a
+// few W tiles and X blocks in L2.
 #include <cuda_bf16.h>
 
 #include "awq_internal.h"
@@ -42,18 +53,21 @@ constexpr int EPI_WARP0 = 16;                          // warps 16-19: TMEM lane
 constexpr int WARP_TMA = 20;
 constexpr int WARP_MMA = 21;
 constexpr int NUM_THREADS = 22 * 32;
-constexpr int X_STAGE_BYTES = SUB_N * SLAB_K * 2;      // 32 KB of fp16 X
+constexpr int PAIR_O = 2 * TILE_O;                     // output rows per CTA pair
+constexpr int X_HALF = SUB_N / 2;                      // tokens of an N = 256 tile per CTA
+constexpr int X_STAGE_BYTES = X_HALF * SLAB_K * 2;     // 16 KB of fp16 X
 constexpr int A_STAGE_BYTES = TILE_O * SLAB_K * 2;     // 16 KB of fp16 dW
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t IDESC = idesc_f16_f32(TILE_O, SUB_N, false);
+constexpr uint32_t IDESC = idesc_f16_f32(PAIR_O, SUB_N, false);   // M = 256 (pair), N = 256
+constexpr uint16_t PAIR_MASK = 0x3;                    // multicast to both CTAs of the pair
 constexpr float MAGIC = 12582912.0f;                   // 1.5 * 2^23: x + MAGIC - MAGIC = rint(x)
 
 // Shared-memory plan, per weight type.  Input stage = W tile, then s / -1/s of
 // the slab (2 x 64 fp32), then the group parameters [1 or 2 groups][128 rows] float4.
 template <bool WBF16>
 struct Plan {
-    static constexpr int XS = WBF16 ? 4 : 3;            // X ring stages
-    static constexpr int AS = 2;                        // dW ring stages
+    static constexpr int XS = 6;                        // X ring stages (two per slab)
+    static constexpr int AS = 3;                        // dW ring stages
     static constexpr int IS = WBF16 ? 3 : 2;            // input ring stages
     static constexpr int W_BYTES = WBF16 ? 16384 : 32768;
     static constexpr int SN_OFF = W_BYTES;
@@ -72,6 +86,11 @@ struct Unit {
     int nsub;
 };
 
+// The pair (cluster) this CTA belongs to, and the number of pairs.
+__device__ __forceinline__ int64_t pair_id() { return blockIdx.x >> 1; }
+__device__ __forceinline__ int64_t pair_count() { return gridDim.x >> 1; }
+
+// OT counts 256-row pair tiles.
 __device__ __forceinline__ Unit decode(int64_t u, const SearchArgs &a, int64_t OT) {
     Unit r;
     r.g = static_cast<int>(u % a.G);
@@ -147,6 +166,7 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
                                               uint64_t *in_empty, uint8_t *a_ring,
                                               uint64_t *a_full, uint64_t *a_empty,
                                               volatile int *abort_flag) {
+    // a_full lives in the leader CTA and counts the producer warps of both CTAs.
     using P = Plan<WBF16>;
     const int t = threadIdx.x;          // 0..511
     const int r = t >> 2, qc = t & 3;   // row in tile, 16-column quarter of the 64-wide slab
@@ -154,14 +174,18 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
     const int jq = a.gs == 32 ? (qc >> 1) : 0;   // which of the slab's groups (stage holds [groups][128 rows])
     const int64_t nK = a.I / SLAB_K;
     uint32_t it = 0;
-    for (int64_t u = blockIdx.x; u < U; u += gridDim.x) {
+    for (int64_t u = pair_id(); u < U; u += pair_count()) {
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
             const uint32_t is = it % P::IS, as = it % P::AS;
             if (!mbar_wait(&in_full[is], (it / P::IS) & 1u, abort_flag)) return;
-            if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag)) return;
             const uint8_t *in = in_ring + is * P::IN_STAGE;
             uint8_t *dst = a_ring + as * A_STAGE_BYTES;
+            // Read all of this thread's inputs of the slab (16 weights, their s and
+            // -1/s, the group parameters), then hand the input stage back at once so
+            // the next slab's copy can land while this one is computed.
             const float4 prm = reinterpret_cast<const float4 *>(in + P::QP_OFF)[jq * TILE_O + r];
+            float w[2][8];
+            float4 sv[2][4];
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 // Quarters 2-3 take their two 8-column chunks in the opposite order, so
@@ -169,38 +193,43 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
                 const int c = cc ^ (qc >> 1);
                 const int ch = qc * 2 + c;                 // 16-byte chunk within the 128-byte row
                 const float *s_sm = reinterpret_cast<const float *>(in + P::SN_OFF) + ch * 8;
-                float w[8];
                 if constexpr (WBF16) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(in + sw128_offset(r, ch));
                     const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        w[2 * k] = __uint_as_float(u4[k] << 16);
-                        w[2 * k + 1] = __uint_as_float(u4[k] & 0xFFFF0000u);
+                        w[cc][2 * k] = __uint_as_float(u4[k] << 16);
+                        w[cc][2 * k + 1] = __uint_as_float(u4[k] & 0xFFFF0000u);
                     }
                 } else {
                     const uint8_t *sub = in + (ch >> 2) * 16384;   // 32-column fp32 sub-tile
                     const int sc = (ch & 3) * 2;                     // its 16-byte chunks
                     const float4 v0 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, sc));
                     const float4 v1 = *reinterpret_cast<const float4 *>(sub + sw128_offset(r, sc + 1));
-                    w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-                    w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+                    w[cc][0] = v0.x; w[cc][1] = v0.y; w[cc][2] = v0.z; w[cc][3] = v0.w;
+                    w[cc][4] = v1.x; w[cc][5] = v1.y; w[cc][6] = v1.z; w[cc][7] = v1.w;
                 }
-                const float4 s0 = *reinterpret_cast<const float4 *>(s_sm);
-                const float4 s1 = *reinterpret_cast<const float4 *>(s_sm + 4);
-                const float4 n0 = *reinterpret_cast<const float4 *>(s_sm + 64);
-                const float4 n1 = *reinterpret_cast<const float4 *>(s_sm + 68);
-                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, ch)) =
-                    dw_chunk8<CLAMP>(w, s0, s1, n0, n1, prm);
+                sv[cc][0] = *reinterpret_cast<const float4 *>(s_sm);
+                sv[cc][1] = *reinterpret_cast<const float4 *>(s_sm + 4);
+                sv[cc][2] = *reinterpret_cast<const float4 *>(s_sm + 64);
+                sv[cc][3] = *reinterpret_cast<const float4 *>(s_sm + 68);
             }
-            // One arrival per warp: every lane's reads and fenced writes are ordered
-            // before lane 0's arrive by the warp barrier.
+            // One arrival per warp: the warp barrier orders every lane's reads
+            // before lane 0's arrive.
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&in_empty[is]);
+            if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag)) return;
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                const int ch = qc * 2 + (cc ^ (qc >> 1));
+                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, ch)) =
+                    dw_chunk8<CLAMP>(w[cc], sv[cc][0], sv[cc][1], sv[cc][2], sv[cc][3], prm);
+            }
+            // One arrival per warp: every lane's fenced writes are ordered before
+            // lane 0's arrive by the warp barrier.
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&in_empty[is]);
-                mbar_arrive(&a_full[as]);
-            }
+            if (lane == 0) mbar_arrive_cluster(cluster_addr(&a_full[as], 0));
         }
     }
 }
@@ -219,9 +248,9 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
 #pragma unroll
     for (int s = 0; s < P::IS; ++s) last[s] = -1;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
+    for (int64_t u = pair_id(); u < U && ok; u += pair_count()) {
         const Unit un = decode(u, a, OT);
-        const int32_t y_w = static_cast<int32_t>(un.ot * TILE_O);
+        const int32_t y_w = static_cast<int32_t>(un.ot * PAIR_O + cluster_ctarank() * TILE_O);
         const int64_t nG = a.I / a.gs;
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
             const uint32_t st = it % P::IS;
@@ -252,18 +281,21 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
         if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / P::IS) & 1));
 }
 
-// Lane 0 of the TMA warp: X tiles for the MMA.
+// Lane 0 of the TMA warp: this CTA's half (128 tokens) of each X tile for the
+// pair MMA.  The leader expects the bytes of both halves on its x_full; the
+// peer's copy completes on the leader's barrier too.  Before refilling a stage
+// each CTA waits for its own x_empty, which the leader's MMA commit signals in
+// both CTAs.  (A copy still in flight when the loop stops was issued at least a
+// full wait bound earlier, so it has landed before the CTA exits.)
 template <int XS>
 __device__ __forceinline__ void x_loader(const SearchArgs &a, const CUtensorMap *xmap, int64_t OT,
                                          int64_t U, uint8_t *x_ring, uint64_t *x_full,
                                          uint64_t *x_empty, volatile int *abort_flag) {
     const int64_t nK = a.I / SLAB_K;
+    const uint32_t rank = cluster_ctarank();
     uint32_t it = 0;
-    int64_t last[XS];
-#pragma unroll
-    for (int s = 0; s < XS; ++s) last[s] = -1;
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
+    for (int64_t u = pair_id(); u < U && ok; u += pair_count()) {
         const Unit un = decode(u, a, OT);
         for (int64_t kb = 0; kb < nK && ok; ++kb) {
             for (int h = 0; h < un.nsub; ++h, ++it) {
@@ -272,19 +304,13 @@ __device__ __forceinline__ void x_loader(const SearchArgs &a, const CUtensorMap 
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(&x_full[stage], X_STAGE_BYTES);
-                tma_load_2d(x_ring + stage * X_STAGE_BYTES, xmap, &x_full[stage],
-                            static_cast<int32_t>(kb * SLAB_K),
-                            static_cast<int32_t>(un.tb * TILE_N + h * SUB_N));
-#pragma unroll
-                for (int s = 0; s < XS; ++s)
-                    if (s == static_cast<int>(stage)) last[s] = it;
+                if (rank == 0) mbar_arrive_expect_tx(&x_full[stage], 2 * X_STAGE_BYTES);
+                tma_load_2d_pair(x_ring + stage * X_STAGE_BYTES, xmap, cluster_addr(&x_full[stage], 0),
+                                 static_cast<int32_t>(kb * SLAB_K),
+                                 static_cast<int32_t>(un.tb * TILE_N + h * SUB_N + rank * X_HALF));
             }
         }
     }
-#pragma unroll
-    for (int s = 0; s < XS; ++s)
-        if (last[s] >= 0) mbar_wait_drain(&x_full[s], static_cast<uint32_t>((last[s] / XS) & 1));
 }
 
 template <int XS, int AS>
@@ -298,7 +324,7 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
     uint32_t ait = 0, xit = 0, accit = 0;
     const uint32_t x_base = smem_u32(x_ring), a_base = smem_u32(a_ring);
     bool ok = true;
-    for (int64_t u = blockIdx.x; u < U && ok; u += gridDim.x) {
+    for (int64_t u = pair_id(); u < U && ok; u += pair_count()) {
         const Unit un = decode(u, a, OT);
         if (!mbar_wait(acc_empty, (accit & 1u) ^ 1u, abort_flag)) break;
         tc_fence_after();
@@ -320,21 +346,21 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
                 const uint32_t b_addr = x_base + xs * X_STAGE_BYTES;
 #pragma unroll
                 for (int k = 0; k < SLAB_K / 16; ++k) {
-                    umma_f16(tmem_base + static_cast<uint32_t>(h * SUB_N),
-                             sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
-                             IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_f16_pair(tmem_base + static_cast<uint32_t>(h * SUB_N),
+                                  sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32),
+                                  IDESC, (kb > 0 || k > 0) ? 1u : 0u);
                 }
-                umma_commit(&x_empty[xs]);
+                umma_commit_pair(&x_empty[xs], PAIR_MASK);
             }
-            if (ok) umma_commit(&a_empty[as]);
+            if (ok) umma_commit_pair(&a_empty[as], PAIR_MASK);
         }
         if (!ok) break;
-        umma_commit(acc_full);
+        umma_commit_pair(acc_full, PAIR_MASK);
         ++accit;
     }
-    // Wait until every MMA this thread issued has finished before TMEM is freed.
-    umma_commit(drain);
-    mbar_wait_drain(drain, 0);
+    // Both CTAs wait on their drain barrier until every MMA issued here has
+    // finished, before TMEM is freed.
+    umma_commit_pair(drain, PAIR_MASK);
 }
 
 __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, int64_t U, int64_t TB,
@@ -345,7 +371,7 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     uint32_t accit = 0;
-    for (int64_t u = blockIdx.x; u < U; u += gridDim.x, ++accit) {
+    for (int64_t u = pair_id(); u < U; u += pair_count(), ++accit) {
         const Unit un = decode(u, a, OT);
         const bool ok = mbar_wait_sleep(acc_full, accit & 1u, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) return;
@@ -361,8 +387,9 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
             }
         }
         tc_fence_before();
-        mbar_arrive(acc_empty);
-        const int64_t row = un.ot * TILE_O + r;
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(acc_empty, 0));
+        const int64_t row = un.ot * PAIR_O + cluster_ctarank() * TILE_O + r;
         if (row < a.O) a.part[(static_cast<int64_t>(un.g) * TB + un.tb) * a.O + row] = sum;
     }
 }
@@ -391,17 +418,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-    const int64_t OT = (a.O + TILE_O - 1) / TILE_O;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t OT = (a.O + PAIR_O - 1) / PAIR_O;
     const int64_t TB = (a.N + TILE_N - 1) / TILE_N;
     const int64_t U = OT * TB * a.G;
 
+    // Barrier counts.  Leader-only barriers (x_full, a_full, acc_empty) count
+    // arrivals from both CTAs; the peer initialises its copies but never waits
+    // on them.
     if (threadIdx.x == 0) {
         for (int s = 0; s < P::XS; ++s) {
-            mbar_init(&x_full[s], 1);
-            mbar_init(&x_empty[s], 1);
+            mbar_init(&x_full[s], 1);                       // leader's expect_tx; bytes of both halves
+            mbar_init(&x_empty[s], 1);                      // the leader's multicast commit
         }
         for (int s = 0; s < P::AS; ++s) {
-            mbar_init(&a_full[s], NUM_PRODUCER_WARPS);
+            mbar_init(&a_full[s], 2 * NUM_PRODUCER_WARPS);  // producer warps of both CTAs
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < P::IS; ++s) {
@@ -409,14 +440,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&in_empty[s], NUM_PRODUCER_WARPS);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 4 * 32);
+        mbar_init(acc_empty, 2 * 4);                        // epilogue warps of both CTAs
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == WARP_MMA) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if (warp == WARP_TMA && lane == 0) {
         tma_prefetch_desc(&maps.x);
@@ -424,8 +455,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_prefetch_desc(&maps.sn);
         tma_prefetch_desc(&maps.qp);
     }
+    // Both CTAs' barriers are initialised, and TMEM allocated, before either
+    // CTA signals the other.
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
@@ -441,7 +474,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             input_loader<WBF16>(a, maps, OT, U, in_ring, in_full, in_empty, abort_flag);
         __syncwarp();
     } else {
-        if (lane == 0)
+        if (lane == 0 && rank == 0)
             mma_role<P::XS, P::AS>(a, OT, U, tmem_base, x_ring, a_ring, x_full, x_empty, a_full,
                                    a_empty, acc_full, acc_empty, drain, abort_flag);
         __syncwarp();
@@ -449,10 +482,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     tc_fence_before();
     __syncthreads();
+    // Every pair MMA has finished (the leader's last commit reaches both CTAs)
+    // before TMEM is freed, and neither CTA leaves while the other may still
+    // signal its barriers or read its shared memory.
+    if (warp == WARP_MMA && lane == 0) mbar_wait_drain(drain, 0);
+    __syncwarp();
+    cluster_sync_all();
     if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err, DEV_ERR_TIMEOUT);
     if (warp == WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
@@ -470,12 +509,33 @@ cudaError_t launch_search_t(const SearchArgs &a, const SearchMaps &maps, int num
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
-    const int64_t OT = (a.O + TILE_O - 1) / TILE_O;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // Persistent: as many pairs as can be resident at once (one CTA per SM).
+    static int max_pairs[64] = {};
+    int pairs_fit = (dev >= 0 && dev < 64) ? max_pairs[dev] : 0;
+    if (pairs_fit == 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+        e = cudaOccupancyMaxActiveClusters(&pairs_fit, search_kernel<WBF16, CLAMP>, &cfg);
+        if (e != cudaSuccess) return e;
+        if (pairs_fit < 1) return cudaErrorInvalidConfiguration;
+        if (dev >= 0 && dev < 64) max_pairs[dev] = pairs_fit;
+    }
+    const int64_t OT = (a.O + PAIR_O - 1) / PAIR_O;
     const int64_t TB = (a.N + TILE_N - 1) / TILE_N;
     const int64_t U = OT * TB * a.G;
-    const int grid = static_cast<int>(U < num_sms ? U : num_sms);
-    search_kernel<WBF16, CLAMP><<<grid, NUM_THREADS, smem, st>>>(maps, a);
-    return cudaGetLastError();
+    const int64_t pairs = U < pairs_fit ? U : pairs_fit;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    return cudaLaunchKernelEx(&cfg, search_kernel<WBF16, CLAMP>, maps, a);
 }
 
 }  // namespace

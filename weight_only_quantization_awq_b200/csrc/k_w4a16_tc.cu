@@ -72,13 +72,14 @@ __global__ void __launch_bounds__(256) xs_absmax_kernel(const uint16_t *__restri
     }
 }
 
-// Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero max).
+// Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero max),
+// clamped to [-125, 125] so that 2^k and 2^-k stay normal floats.
 __device__ __forceinline__ int pow2_exp(float mx, int top) {
     if (!(mx > 0.0f) || isinf(mx)) return 0;
     int e;
     frexpf(mx, &e);                                   // mx = f * 2^e, f in [0.5, 1)
     const int k = e - top;
-    return k < -100 ? -100 : (k > 100 ? 100 : k);
+    return k < -125 ? -125 : (k > 125 ? 125 : k);
 }
 
 // words: [0] max |xs| bits, [1] kx, [2] max |Delta| bits, [3] kd.
@@ -295,7 +296,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int64_t m0 = mt * TC_TOKENS;
         const int mcount = static_cast<int>(a.M - m0 < a.n_tile ? a.M - m0 : a.n_tile);
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-        const float yscale = ldexpf(1.0f, static_cast<int>(a.words[1]) + static_cast<int>(a.words[3]));
+        // y = accumulator * 2^kx * 2^kd, two normal factors (their product can be subnormal)
+        const float ysx = ldexpf(1.0f, static_cast<int>(a.words[1]));
+        const float ysd = ldexpf(1.0f, static_cast<int>(a.words[3]));
         if (__all_sync(0xffffffffu, got)) {
             for (int c = 0; c < a.n_tile; c += 16) {
                 uint32_t rv[16];
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int k = 0; k < 16; ++k) {
                     const int n = c + k;
                     if (n < mcount && erow_ok) {
-                        const float v = __uint_as_float(rv[k]) * yscale;
+                        const float v = (__uint_as_float(rv[k]) * ysx) * ysd;
                         if (a.splits == 1)
                             a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
                         else
