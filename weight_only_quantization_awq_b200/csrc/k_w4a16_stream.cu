@@ -182,6 +182,7 @@ __global__ void __launch_bounds__(GvShape<MT>::NW * 32, 1) w4a16_gemv_kernel(con
     // (the loop bound is uniform per warp: the shuffles below need all 32 lanes)
     constexpr int KOFF = 15;                         // max |xs| lands in [2^(KOFF-1), 2^KOFF)
     for (int tb = 0; tb < ntask; tb += GV_THREADS) {
+        if (tb + warp * 32 >= ntask) break;          // no task left for this warp (warp-uniform)
         const int task = tb + threadIdx.x;
         const bool live = task < ntask;
         const int wd = task & 3, ch = task >> 2;
