@@ -26,7 +26,8 @@
 //               layout the MMA reads, arrive on the leader's a_full.
 //   warps 16-19 epilogue: tcgen05.ld of the CTA's 128 x 512 fp32 accumulator
 //               (lane = output row), square-and-sum per row, one fp32 partial
-//               per (grid point, token block, row).
+//               per (grid point, token block, row); each 256-column half is
+//               handed back to the MMA as soon as it has been read.
 //   warp 20     TMA: lane 0 streams this CTA's half of the X tiles (128 tokens x
 //               64 channels, fp16 copy of X scaled by a power of two) into the X
 //               ring, counted on the leader's x_full; lane 1 streams each slab's
@@ -73,7 +74,7 @@ struct Plan {
     static constexpr int SN_OFF = W_BYTES;
     static constexpr int QP_OFF = SN_OFF + 512;
     static constexpr int IN_STAGE = ((QP_OFF + 4096) + 1023) / 1024 * 1024;
-    static constexpr int NUM_BARS = 2 * XS + 2 * AS + 2 * IS + 3;
+    static constexpr int NUM_BARS = 2 * XS + 2 * AS + 2 * IS + 5;
     static constexpr int SMEM_BYTES =
         1024 + XS * X_STAGE_BYTES + AS * A_STAGE_BYTES + IS * IN_STAGE + NUM_BARS * 8 + 16;
 };
@@ -321,13 +322,12 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
                                          uint64_t *acc_empty, uint64_t *drain,
                                          volatile int *abort_flag) {
     const int64_t nK = a.I / SLAB_K;
-    uint32_t ait = 0, xit = 0, accit = 0;
+    uint32_t ait = 0, xit = 0;
+    uint32_t hit[2] = {0u, 0u};                    // units that have used each accumulator half
     const uint32_t x_base = smem_u32(x_ring), a_base = smem_u32(a_ring);
     bool ok = true;
     for (int64_t u = pair_id(); u < U && ok; u += pair_count()) {
         const Unit un = decode(u, a, OT);
-        if (!mbar_wait(acc_empty, (accit & 1u) ^ 1u, abort_flag)) break;
-        tc_fence_after();
         for (int64_t kb = 0; kb < nK && ok; ++kb, ++ait) {
             const uint32_t as = ait % AS;
             if (!mbar_wait(&a_full[as], (ait / AS) & 1u, abort_flag)) {
@@ -337,6 +337,15 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
             tc_fence_after();
             const uint32_t a_addr = a_base + as * A_STAGE_BYTES;
             for (int h = 0; h < un.nsub; ++h, ++xit) {
+                // each 256-column half of the accumulator is waited for separately, so
+                // this unit starts on half 0 while the epilogue still drains half 1
+                if (kb == 0) {
+                    if (!mbar_wait(&acc_empty[h], (hit[h] & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
                 const uint32_t xs = xit % XS;
                 if (!mbar_wait(&x_full[xs], (xit / XS) & 1u, abort_flag)) {
                     ok = false;
@@ -351,12 +360,12 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
                                   IDESC, (kb > 0 || k > 0) ? 1u : 0u);
                 }
                 umma_commit_pair(&x_empty[xs], PAIR_MASK);
+                if (kb == nK - 1) umma_commit_pair(&acc_full[h], PAIR_MASK);
             }
             if (ok) umma_commit_pair(&a_empty[as], PAIR_MASK);
         }
         if (!ok) break;
-        umma_commit_pair(acc_full, PAIR_MASK);
-        ++accit;
+        for (int h = 0; h < un.nsub; ++h) ++hit[h];
     }
     // Both CTAs wait on their drain barrier until every MMA issued here has
     // finished, before TMEM is freed.
@@ -370,14 +379,14 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
     const int lane = threadIdx.x & 31;
     const int r = quad * 32 + lane;
     const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-    uint32_t accit = 0;
-    for (int64_t u = pair_id(); u < U; u += pair_count(), ++accit) {
+    uint32_t hit[2] = {0u, 0u};                    // units that have used each accumulator half
+    for (int64_t u = pair_id(); u < U; u += pair_count()) {
         const Unit un = decode(u, a, OT);
-        const bool ok = mbar_wait_sleep(acc_full, accit & 1u, abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) return;
-        tc_fence_after();
         float sum = 0.0f;
         for (int h = 0; h < un.nsub; ++h) {
+            const bool ok = mbar_wait_sleep(&acc_full[h], hit[h] & 1u, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) return;
+            tc_fence_after();
 #pragma unroll 1
             for (int c = 0; c < SUB_N / 32; ++c) {
                 float v[32];
@@ -385,10 +394,12 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
 #pragma unroll
                 for (int k = 0; k < 32; ++k) sum = __fmaf_rn(v[k], v[k], sum);
             }
+            // this half may be overwritten by the next unit as soon as both CTAs' epilogues have read it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(cluster_addr(&acc_empty[h], 0));
+            ++hit[h];
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(cluster_addr(acc_empty, 0));
         const int64_t row = un.ot * PAIR_O + cluster_ctarank() * TILE_O + r;
         if (row < a.O) a.part[(static_cast<int64_t>(un.g) * TB + un.tb) * a.O + row] = sum;
     }
@@ -411,9 +422,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t *a_empty = a_full + P::AS;
     uint64_t *in_full = a_empty + P::AS;
     uint64_t *in_empty = in_full + P::IS;
-    uint64_t *acc_full = in_empty + P::IS;
-    uint64_t *acc_empty = acc_full + 1;
-    uint64_t *drain = acc_empty + 1;
+    uint64_t *acc_full = in_empty + P::IS;         // [2]: one per 256-column accumulator half
+    uint64_t *acc_empty = acc_full + 2;            // [2]
+    uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -439,8 +450,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&in_full[s], 1);
             mbar_init(&in_empty[s], NUM_PRODUCER_WARPS);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 2 * 4);                        // epilogue warps of both CTAs
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&acc_full[h], 1);
+            mbar_init(&acc_empty[h], 2 * 4);                // epilogue warps of both CTAs
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
