@@ -15,8 +15,8 @@
 // forms and holds 128 (its own rows of dW), and N = 256 tokens per
 // instruction, of which each CTA stages 128 (half of each X tile).  Each CTA's
 // TMEM receives its 128 rows x all 512 tokens of the unit.  So each SM streams
-// half of the X tiles a single-CTA MMA of the same shape would need: X re-reads
-// from L2 are what bound the single-CTA form of this kernel.
+// and stores half of the X tiles a single-CTA MMA of the same shape would need
+// (the tensor cores of the pair read each other's halves).
 //
 // Warp roles (704 threads per CTA):
 //   warps 0-15  dW producers (16 columns of one row per thread): read one slab's
