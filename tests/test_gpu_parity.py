@@ -272,3 +272,20 @@ def test_linear_w4a16_activation_range(awq, M, pattern):
         assert np.all(y == 0.0)
     else:
         check_apply(got, y_ref)
+
+
+@pytest.mark.parametrize("M,I", [(3, 24576), (4, 24576), (4, 40960), (2, 49152), (1, 49152)])
+def test_linear_w4a16_widest_inputs(awq, M, I):
+    """Input widths at the top of the supported range: 2-4 tokens this wide do
+    not fit the streaming kernel's shared activation table and take the fallback
+    decode kernel (two tokens per pass at 24576 columns, one per pass at 40960
+    and 49152); in = 49152 is the largest width accepted."""
+    O, gs = 96, 128
+    W, X = small_layer(O, I, 16, seed=M + I)
+    p = oracle.pack_int4(W, oracle.act_stats(X), 0.5, 1.0, gs, 1)
+    x = apply_activations(M, I, seed=M + 7)
+    y_ref = oracle.linear_w4a16(x, p["qweight"], p["scales"], p["zeros"], p["s16"], gs)
+    got = awq.awq_linear_w4a16(
+        dev(x), dev(p["qweight"].view(np.int32)), dev(p["scales"].view(np.float16)),
+        dev(p["zeros"].view(np.int32)), dev(p["s16"].view(np.float16)), gs)
+    check_apply(got, y_ref)

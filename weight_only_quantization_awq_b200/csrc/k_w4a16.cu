@@ -209,6 +209,7 @@ cudaError_t launch_w4a16(const uint16_t *x, int64_t M, int64_t I, int64_t O,
 #define AWQ_DEC(MT)                                                                      \
     return z ? launch_decode<MT, true>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st) \
              : launch_decode<MT, false>(x, M, I, O, qweight, scales, zeros, s16, gs, y, st)
+    if (2 * per_token > 227 * 1024) AWQ_DEC(1);      // wide inputs: one token's activations per pass
     if (M <= 2 || 4 * per_token > 227 * 1024) AWQ_DEC(2);
     if (M <= 4 || 8 * per_token > 227 * 1024) AWQ_DEC(4);
     AWQ_DEC(8);

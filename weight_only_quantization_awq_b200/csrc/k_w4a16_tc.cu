@@ -21,9 +21,11 @@
 //                   fp32 accumulate in TMEM).
 //     warps 0-3     epilogue: tcgen05.ld of the accumulator; with one K split
 //                   y is written directly, otherwise each split adds its fp32
-//                   partial into a zeroed fp32 tile with red.global.add (the order
-//                   of those adds across splits is not fixed) and the last CTA of
-//                   the tile (counter) converts the tile to bf16.
+//                   partial, still unscaled (normal-range values, untouched by the
+//                   atomic's flush of subnormals), into a zeroed fp32 tile with
+//                   red.global.add (the order of those adds across splits is not
+//                   fixed) and the last CTA of the tile (counter) applies the
+//                   power-of-two scales and converts the tile to bf16.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -307,11 +309,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int k = 0; k < 16; ++k) {
                     const int n = c + k;
                     if (n < mcount && erow_ok) {
-                        const float v = (__uint_as_float(rv[k]) * ysx) * ysd;
-                        if (a.splits == 1)
-                            a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-                        else
-                            atomicAdd(a.acc32 + (m0 + n) * a.O + eo, v);   // result unused: red.global.add
+                        const float acc = __uint_as_float(rv[k]);
+                        if (a.splits == 1) {
+                            a.y[(m0 + n) * a.O + eo] =
+                                __bfloat16_as_ushort(__float2bfloat16_rn((acc * ysx) * ysd));
+                        } else {
+                            // split-K partials meet unscaled: they lie in the normal range,
+                            // where the float atomic's flush of subnormals cannot bite
+                            atomicAdd(a.acc32 + (m0 + n) * a.O + eo, acc);   // result unused: red.global.add
+                        }
                     }
                 }
             }
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll 8
                     for (int n = 0; n < mcount; ++n)
                         a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(
-                            __float2bfloat16_rn(__ldcg(a.acc32 + (m0 + n) * a.O + eo)));
+                            __float2bfloat16_rn((__ldcg(a.acc32 + (m0 + n) * a.O + eo) * ysx) * ysd));
                 }
             }
         }
