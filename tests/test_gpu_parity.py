@@ -121,6 +121,9 @@ SEARCH_CASES = [
     (128, 512, 1024, 32, 0, None, "bf16", "f32"),
     (300, 640, 513, 128, 1, CLIP_GRID, "bf16", "bf16"),  # 1-token tail block
     (16, 128, 2048, 128, 0, CLIP_GRID[:3], "bf16", "bf16"),
+    (1, 64, 64, 32, 1, CLIP_GRID[:2], "bf16", "bf16"),  # one row, one slab
+    (3, 64, 5, 64, 0, None, "f32", "bf16"),              # one slab: the first slab is the last
+    (257, 192, 257, 64, 1, None, "bf16", "bf16"),       # one row into a second pair tile
 ]
 
 
