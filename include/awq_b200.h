@@ -90,8 +90,11 @@ awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in,
  *             AWQ_ASYM Delta = (max w - min w)/15, z = clamp(rint(-min/Delta), 0, 15),
  *                      q = clamp(rint(w/Delta) + z, 0, 15), value (q - z)*Delta.
  * W         : [out, in] device, fp32 or bf16 (w_dtype).
- * X         : [N, in] device, fp32 or bf16 (x_dtype); fp32 X is rounded to bf16
- *             for the tensor-core contraction.
+ * X         : [N, in] device, fp32 or bf16 (x_dtype).  The tensor-core
+ *             contraction reads an fp16 copy of X scaled by one power of two
+ *             (largest magnitude in [2^14, 2^15)), so bf16 values down to 2^-28
+ *             of the maximum are exact and fp32 values are rounded to fp16's
+ *             11-bit significand; the losses are rescaled exactly.
  * sX        : [in] fp32 device (from awq_act_stats).
  * alpha     : [n_alpha] host, 1 <= n_alpha <= 64, each in [0, 1].
  * clip      : [n_clip] host or NULL, 0 <= n_clip <= 64, each in (0, 1].
@@ -143,8 +146,9 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in,
  * Ordering: the M <= 4 kernel is launched with programmatic stream
  * serialisation, so its blocks may start while the preceding kernel on
  * `stream` is still running; until that kernel has completed they only ask L2
- * to prefetch qweight, scales and zeros (a hint that reads nothing into the
- * SM), and every read of an argument, and the write of y, happens after it.
+ * to prefetch qweight, scales, zeros, s16 and x (a hint that reads nothing
+ * into the SM), and every read of an argument, and the write of y, happens
+ * after it.
  */
 awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
                               const uint32_t *qweight, const uint16_t *scales,
