@@ -441,7 +441,7 @@ def oracle_step(W_np, X_np, rows):
     return res
 
 
-def cpu_baseline(W_np, X_np, rows_per_core=16):
+def cpu_baseline(W_np, X_np, rows_per_core=48):
     import numpy as np
     cores = _oracle_threads()
     O = W_np.shape[0]
