@@ -6,6 +6,7 @@ the computation runs in the library's kernels.  The functions carry the C
 names:
 
     awq_act_stats(X)                         -> s_X = mean |X| per input channel
+    awq_act_stats_noalloc(X)                 -> the same without any device allocation
     awq_search_layer(W, X, sX, ...)          -> losses over the alpha (and clip) grid, argmin
     awq_pack_int4(W, sX, alpha, clip, ...)   -> packed INT4 codes, fp16 scales, zeros, s
     awq_linear_w4a16(x, packed...)           -> y = (x / s) @ dequant(W)^T
