@@ -45,8 +45,10 @@ def test_act_stats_noalloc_matches_allocating_entry_point():
                                        out.data_ptr(), stream)
         assert st == 0, lib.awq_last_error().decode()
         ref = awq.awq_act_stats(Xd)
+        via_binding = awq.awq_act_stats_noalloc(Xd)
         torch.cuda.synchronize()
         assert torch.equal(out, ref)
+        assert torch.equal(via_binding, ref)
 
     # beyond the fixed buffer (ceil(N/128) * in > 2^20): refused, nothing enqueued
     big = torch.empty((128 * 129, 8192), dtype=torch.bfloat16, device="cuda")

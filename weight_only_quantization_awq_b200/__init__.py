@@ -132,6 +132,20 @@ def awq_act_stats(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.Tensor | 
     return out
 
 
+def awq_act_stats_noalloc(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.Tensor | None = None):
+    """awq_act_stats through the library's allocation-free entry point (its fp64
+    partials live in a fixed device buffer; ceil(N / 128) * in <= 1,048,576).
+    Pass `out` ([in] fp32 device) to allocate nothing at all."""
+    _dev(X, "X")
+    N, inp = X.shape
+    if out is None:
+        out = torch.empty(inp, dtype=torch.float32, device=X.device)
+    _check("awq_act_stats_noalloc",
+           lib.awq_act_stats_noalloc(X.data_ptr(), _dtype_code(X), N, inp, float(clamp_min),
+                                     out.data_ptr(), _stream(X)))
+    return out
+
+
 def awq_search_layer(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, group_size: int = 128,
                      w_bit: int = 4, quant="sym", alpha=ALPHA_GRID_20, clip=None,
                      loss_row: bool = False):
