@@ -150,10 +150,64 @@ def test_quant_group_asym_brute_force(gs):
         assert z == _brute_nearest(float(np.float32(-mn) / d), 0, 15)
         for k in range(gs):
             t = np.float32(w[k]) / d
-            assert q[k] == _brute_nearest(float(t) + z, 0, 15) or \
-                q[k] == min(max(_brute_nearest(float(t), -100, 100) + z, 0), 15)
+            # one rule: the nearest representable offset q - z to the fp32 quotient,
+            # ties to the even offset (rint(t) + z, then the clamp)
+            assert q[k] == _brute_nearest(float(t), -z, 15 - z) + z
             assert abs(float(w[k]) - (q[k] - z) * float(d)) <= float(d) * (1 + 1e-6)
         assert q[np.argmin(w)] <= 1 and q[np.argmax(w)] >= 14
+
+
+def test_quant_group_asym_tie_with_odd_zero_point():
+    """Range [-3, 12]: Delta = 1 and z = 3 (odd).  Half-integer quotients round
+    to the even offset q - z (2.5 -> 2 -> code 5; -0.5 -> 0 -> code 3), not to
+    the even code (rounding t + z would give 6 and 2)."""
+    g = np.array([12.0, -3.0, 2.5, -0.5, 0.5, 1.5, 4.5] + [1.0] * 121, np.float32)
+    q, d, z = oracle.quant_group(g, oracle.ASYM)
+    assert d == np.float32(1.0) and z == 3
+    assert list(q[:7]) == [15, 0, 5, 3, 3, 5, 7]
+
+
+def test_quant_group_asym_clip_hand_cases():
+    """Clip r scales both bounds before Delta and z are formed; values beyond
+    the clipped bounds saturate.  Range [-3, 12] at r = 0.5: bounds [-1.5, 6],
+    Delta = 7.5 / 15 = 0.5, z = rint(1.5 / 0.5) = 3.  Clipping only the maximum
+    would give Delta = 0.6, z = 5; a zero point from the unclipped minimum
+    would give z = 6."""
+    g = np.array([12.0, -3.0, 0.25, 0.75, 2.5, -0.5, 6.0, -1.5, 6.2, -1.8] + [1.0] * 118,
+                 np.float32)
+    q, d, z = oracle.quant_group(g, oracle.ASYM, clip=0.5)
+    assert d == np.float32(0.5) and z == 3
+    #            12  -3  .25 .75 2.5 -.5  6  -1.5 6.2 -1.8
+    assert list(q[:10]) == [15, 0, 3, 5, 8, 2, 15, 0, 15, 0]
+    # r = 0.25: bounds [-0.75, 3], Delta = 0.25, z = 3; 0.25 -> t = 1 -> code 4
+    q, d, z = oracle.quant_group(g, oracle.ASYM, clip=0.25)
+    assert d == np.float32(0.25) and z == 3
+    assert list(q[:6]) == [15, 0, 4, 6, 13, 1]
+
+
+@pytest.mark.parametrize("r", [0.9, 0.5])
+def test_quant_group_asym_clip_fp32_and_enumeration(r):
+    """Random groups at clip r: Delta and z bit-exact against the fp32 formulas
+    (r applied to each bound in fp64 and rounded once, then one fp32 subtract and
+    one fp32 divide); every code is the nearest representable offset after
+    clipping, found by enumeration, ties to the even offset; elements beyond the
+    clipped bounds saturate to 0 or 15."""
+    g = rng(70 + int(r * 10))
+    for trial in range(60):
+        w = (g.standard_normal(128) * 0.05 + g.uniform(-0.03, 0.03)).astype(np.float32)
+        q, d, z = oracle.quant_group(w, oracle.ASYM, clip=r)
+        mxr = np.float32(np.float64(w.max()) * r)
+        mnr = np.float32(np.float64(w.min()) * r)
+        want_d = np.float32(mxr - mnr) / np.float32(15.0)
+        assert d == want_d
+        want_z = int(min(max(np.rint(np.float32(-mnr) / want_d), 0.0), 15.0))
+        assert z == want_z
+        for k in range(128):
+            t = float(np.float32(w[k]) / d)
+            assert q[k] == _brute_nearest(t, -z, 15 - z) + z
+            if w[k] > mxr + d or w[k] < mnr - d:
+                assert q[k] in (0, 15)
+        assert q[np.argmax(w)] == 15 and q[np.argmin(w)] == 0
 
 
 def test_quant_group_scale_invariance():
@@ -304,6 +358,63 @@ def test_search_brute_force_argmin_and_invariants():
     assert res["loss"][0] == pytest.approx(rtn, rel=1e-12)
     assert res["loss"][len(alpha)] == res["loss"][res["best_alpha"]]
     assert res["best_clip"] == int(np.argmin(res["loss"][len(alpha):]))
+
+
+def _enum_quant_layer(W, s, gs, qt, clip):
+    """Codes of Q(W*s) found by enumeration: per group the bounds (times clip)
+    give Delta (and z); each element takes the nearest representable offset to
+    its fp32 quotient, ties to the even offset."""
+    Wf = oracle.as_f32(W)
+    O, I = Wf.shape
+    c = np.zeros((O, I), np.int64)
+    d = np.zeros((O, I // gs), np.float32)
+    z = np.zeros((O, I // gs), np.int64)
+    for o in range(O):
+        for j in range(I // gs):
+            wp = (Wf[o, j * gs:(j + 1) * gs] * s[j * gs:(j + 1) * gs]).astype(np.float32)
+            if qt == oracle.SYM:
+                a = np.float32(np.float64(np.abs(wp).max()) * clip)
+                dd, zz, lo, hi = np.float32(a) / np.float32(7.0), 0, -8, 7
+            else:
+                mxr = np.float32(np.float64(wp.max()) * clip)
+                mnr = np.float32(np.float64(wp.min()) * clip)
+                dd = np.float32(mxr - mnr) / np.float32(15.0)
+                zz = int(min(max(np.rint(np.float32(-mnr) / dd), 0.0), 15.0))
+                lo, hi = -zz, 15 - zz
+            d[o, j], z[o, j] = dd, zz
+            for k in range(gs):
+                c[o, j * gs + k] = _brute_nearest(float(np.float32(wp[k]) / dd), lo, hi) + zz
+    return c, d, z
+
+
+def test_search_asym_clip_grid_brute_force():
+    """Asymmetric search with a clip grid on a tiny non-square layer: every
+    alpha-phase and clip-phase loss equals the brute-force loss over codes found
+    by enumeration; alpha* and r* are the first minimisers; loss(r = 1.0) equals
+    loss(alpha*)."""
+    O, I, N, gs = 3, 64, 9, 32
+    W, X = small_layer(O, I, N, wdtype="f32", xdtype="f32", seed=71, n_outliers=2, outlier=25.0)
+    sX = oracle.act_stats(X)
+    alpha = ALPHA_GRID[::5]
+    clip = CLIP_GRID[::2]
+    res = oracle.search_layer(W, X, sX, gs, oracle.ASYM, alpha, clip=clip)
+    ref = []
+    for a in alpha:
+        s = oracle.scale_vector(sX, a)
+        c, d, z = _enum_quant_layer(W, s, gs, oracle.ASYM, 1.0)
+        ref.append(_brute_loss_rows(W, X, s, gs, c, d, z).sum() / (N * O))
+    assert np.allclose(res["loss"][:len(alpha)], ref, rtol=1e-12)
+    ba = int(np.argmin(ref))
+    assert res["best_alpha"] == ba
+    s = oracle.scale_vector(sX, alpha[ba])
+    ref_c = []
+    for r in clip:
+        c, d, z = _enum_quant_layer(W, s, gs, oracle.ASYM, float(r))
+        ref_c.append(_brute_loss_rows(W, X, s, gs, c, d, z).sum() / (N * O))
+    assert np.allclose(res["loss"][len(alpha):], ref_c, rtol=1e-12)
+    assert res["best_clip"] == int(np.argmin(ref_c))
+    assert res["loss"][len(alpha)] == res["loss"][ba]          # clip[0] = 1.0
+    assert len(set(np.round(ref_c, 15))) > 2                   # the clip grid changes the loss
 
 
 def test_search_first_minimum_on_ties():
