@@ -52,14 +52,18 @@ def _load():
         lib.orc_stats_chunk.restype = I
         lib.orc_act_stats.argtypes = [P, i64, i64, F, P]
         lib.orc_scale_vector.argtypes = [P, i64, D, P]
-        lib.orc_quant_group.argtypes = [P, I, I, D, P, P, P]
-        lib.orc_quant_layer.argtypes = [P, i64, i64, P, I, I, D, P, P, P]
+        lib.orc_quant_group.argtypes = [P, I, I, I, D, P, P, P]
+        lib.orc_quant_layer.argtypes = [P, i64, i64, P, I, I, I, D, P, P, P, P]
         lib.orc_layer_loss_rows.argtypes = [P, i64, i64, P, i64, P, I, P, P, P, P, i64, P]
         lib.orc_layer_loss_rows.restype = D
-        lib.orc_search_layer.argtypes = [P, i64, i64, P, i64, P, I, I, P, I, P, I,
+        lib.orc_search_layer.argtypes = [P, i64, i64, P, i64, P, I, I, I, P, I, P, I,
                                          P, i64, P, P, P, P]
-        lib.orc_pack_int4.argtypes = [P, i64, i64, P, D, D, I, I, P, P, P, P, P]
+        lib.orc_search_points.argtypes = [P, i64, i64, P, i64, P, I, I, I, P, P, I,
+                                          P, i64, P, P, P]
+        lib.orc_group_clip.argtypes = [P, i64, i64, P, i64, P, D, I, I, I, P, I, P, P]
+        lib.orc_pack_int4.argtypes = [P, i64, i64, P, D, D, P, I, I, I, P, P, P, P, P]
         lib.orc_linear_w4a16.argtypes = [P, i64, i64, i64, P, P, P, P, I, P]
+        lib.orc_fold_scale.argtypes = [P, i64, i64, P, I, P]
         _lib = lib
     return _lib
 
@@ -94,27 +98,45 @@ def scale_vector(sX: np.ndarray, alpha: float) -> np.ndarray:
     return out
 
 
-def quant_group(wp: np.ndarray, qt: int = SYM, clip: float = 1.0):
+def _check_wbit(w_bit):
+    if w_bit not in (3, 4):
+        raise ValueError(f"w_bit {w_bit} not in (3, 4)")
+    return int(w_bit)
+
+
+def _clip_g(clip_g, O, nG):
+    if clip_g is None:
+        return None
+    c = np.ascontiguousarray(clip_g, np.float64)
+    if c.shape != (O, nG):
+        raise ValueError(f"per-group clip must be [{O}, {nG}]")
+    return c
+
+
+def quant_group(wp: np.ndarray, qt: int = SYM, clip: float = 1.0, w_bit: int = 4):
     """Codes, Delta and zero of one group of already-scaled weights."""
     wp = np.ascontiguousarray(wp, np.float32)
     q = np.empty(wp.shape[0], np.int32)
     d = ctypes.c_float()
     z = ctypes.c_int()
-    _load().orc_quant_group(_p(wp), wp.shape[0], qt, float(clip), _p(q),
+    _load().orc_quant_group(_p(wp), wp.shape[0], qt, _check_wbit(w_bit), float(clip), _p(q),
                             ctypes.byref(d), ctypes.byref(z))
     return q, np.float32(d.value), int(z.value)
 
 
-def quant_layer(W: np.ndarray, s: np.ndarray, gs: int, qt: int = SYM, clip: float = 1.0):
-    """codes [O, I] int8, Delta [O, I/gs] fp32, z [O, I/gs] uint8 of Q(W*s)."""
+def quant_layer(W: np.ndarray, s: np.ndarray, gs: int, qt: int = SYM, clip: float = 1.0,
+                w_bit: int = 4, clip_g=None):
+    """codes [O, I] int8, Delta [O, I/gs] fp32, z [O, I/gs] uint8 of Q(W*s);
+    clip_g [O, I/gs] (optional) gives each group its own clip ratio."""
     W = as_f32(W)
     O, I = W.shape
     s = np.ascontiguousarray(s, np.float32)
     codes = np.empty((O, I), np.int8)
     delta = np.empty((O, I // gs), np.float32)
     zeros = np.empty((O, I // gs), np.uint8)
-    _load().orc_quant_layer(_p(W), O, I, _p(s), gs, qt, float(clip), _p(codes),
-                            _p(delta), _p(zeros))
+    cg = _clip_g(clip_g, O, I // gs)
+    _load().orc_quant_layer(_p(W), O, I, _p(s), gs, qt, _check_wbit(w_bit), float(clip),
+                            _p(cg) if cg is not None else None, _p(codes), _p(delta), _p(zeros))
     return codes, delta, zeros
 
 
@@ -133,7 +155,7 @@ def layer_loss_rows(W, X, s, gs, codes, delta, zeros, rows=None):
     return float(tot), lr
 
 
-def search_layer(W, X, sX, gs, qt, alpha, clip=None, rows=None):
+def search_layer(W, X, sX, gs, qt, alpha, clip=None, rows=None, w_bit=4):
     """Grid search.  Returns dict(loss [G+C] fp64, loss_row [G+C, R] fp64,
     best_alpha, best_clip)."""
     W = as_f32(W)
@@ -154,34 +176,78 @@ def search_layer(W, X, sX, gs, qt, alpha, clip=None, rows=None):
     bc = ctypes.c_int()
     _load().orc_search_layer(
         _p(W), O, I, _p(X), N, _p(np.ascontiguousarray(sX, np.float32)), gs, qt,
-        _p(alpha), G, _p(clip) if C else None, C,
+        _check_wbit(w_bit), _p(alpha), G, _p(clip) if C else None, C,
         _p(rows_arr) if rows_arr is not None else None, R,
         _p(loss), _p(loss_row), ctypes.byref(ba), ctypes.byref(bc))
     return {"loss": loss, "loss_row": loss_row, "best_alpha": int(ba.value),
             "best_clip": int(bc.value)}
 
 
-def pack_int4(W, sX, alpha, clip, gs, qt):
-    """Packed storage at (alpha, clip): dict(qweight u32 [O, I/8], scales f16 bits
-    [O, I/gs] (uint16), zeros u32 [O, ceil(I/gs/8)] or None, s16 f16 bits [I],
-    scales_f32 [O, I/gs])."""
+def search_points(W, X, sX, gs, qt, alpha, clip, rows=None, w_bit=4):
+    """The loss at each listed (alpha[k], clip[k]) point.  Returns dict(loss [n],
+    loss_row [n, R], best)."""
+    W = as_f32(W)
+    X = as_f32(X)
+    O, I = W.shape
+    N = X.shape[0]
+    alpha = np.ascontiguousarray(alpha, np.float64)
+    clip = np.ascontiguousarray(clip, np.float64)
+    if alpha.shape != clip.shape:
+        raise ValueError("alpha and clip must list the same number of points")
+    n = alpha.shape[0]
+    rows_arr = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    R = O if rows_arr is None else rows_arr.shape[0]
+    loss = np.empty(n, np.float64)
+    loss_row = np.empty((n, R), np.float64)
+    best = ctypes.c_int()
+    _load().orc_search_points(
+        _p(W), O, I, _p(X), N, _p(np.ascontiguousarray(sX, np.float32)), gs, qt,
+        _check_wbit(w_bit), _p(alpha), _p(clip), n,
+        _p(rows_arr) if rows_arr is not None else None, R, _p(loss), _p(loss_row),
+        ctypes.byref(best))
+    return {"loss": loss, "loss_row": loss_row, "best": int(best.value)}
+
+
+def group_clip(W, X, sX, alpha, gs, qt, clip, w_bit=4, want_err=False):
+    """Per-group clip search at s = s_X^alpha.  Returns dict(best [O, I/gs]
+    int32 indices into clip, err [O, I/gs, n_clip] fp64 or None)."""
+    W = as_f32(W)
+    X = as_f32(X)
+    O, I = W.shape
+    N = X.shape[0]
+    clip = np.ascontiguousarray(clip, np.float64)
+    best = np.empty((O, I // gs), np.int32)
+    err = np.empty((O, I // gs, clip.shape[0]), np.float64) if want_err else None
+    _load().orc_group_clip(_p(W), O, I, _p(X), N, _p(np.ascontiguousarray(sX, np.float32)),
+                           float(alpha), gs, qt, _check_wbit(w_bit), _p(clip), clip.shape[0],
+                           _p(best), _p(err) if err is not None else None)
+    return {"best": best, "err": err}
+
+
+def pack_int4(W, sX, alpha, clip, gs, qt, w_bit=4, clip_g=None):
+    """Packed storage at (alpha, clip), or at the per-group ratios clip_g
+    [O, I/gs]: dict(qweight u32 [O, I/8], scales f16 bits [O, I/gs] (uint16),
+    zeros u32 [O, ceil(I/gs/8)] or None, s16 f16 bits [I], scales_f32 [O, I/gs])."""
     W = as_f32(W)
     O, I = W.shape
     nG = I // gs
+    cg = _clip_g(clip_g, O, nG)
     qweight = np.empty((O, I // 8), np.uint32)
     scales = np.empty((O, nG), np.uint16)
     zeros = np.empty((O, (nG + 7) // 8), np.uint32) if qt == ASYM else None
     s16 = np.empty(I, np.uint16)
     sf = np.empty((O, nG), np.float32)
     _load().orc_pack_int4(_p(W), O, I, _p(np.ascontiguousarray(sX, np.float32)),
-                          float(alpha), float(clip), gs, qt, _p(qweight), _p(scales),
+                          float(alpha), float(clip), _p(cg) if cg is not None else None,
+                          gs, qt, _check_wbit(w_bit), _p(qweight), _p(scales),
                           _p(zeros) if zeros is not None else None, _p(s16), _p(sf))
     return {"qweight": qweight, "scales": scales, "zeros": zeros, "s16": s16,
             "scales_f32": sf}
 
 
 def linear_w4a16(x, qweight, scales, zeros, s16, gs):
-    """y [M, O] fp64 of the W4A16 linear on packed storage."""
+    """y [M, O] fp64 of the W4A16 linear on packed storage (s16 None: x is
+    already divided by s)."""
     x = as_f32(x)
     M, I = x.shape
     O = qweight.shape[0]
@@ -190,5 +256,20 @@ def linear_w4a16(x, qweight, scales, zeros, s16, gs):
         _p(x), M, I, O, _p(np.ascontiguousarray(qweight, np.uint32)),
         _p(np.ascontiguousarray(scales, np.uint16)),
         _p(np.ascontiguousarray(zeros, np.uint32)) if zeros is not None else None,
-        _p(np.ascontiguousarray(s16, np.uint16)), gs, _p(y))
+        _p(np.ascontiguousarray(s16, np.uint16)) if s16 is not None else None, gs, _p(y))
     return y
+
+
+def fold_scale(P, s16, out_bf16=True):
+    """P [R, C] (fp32, or bf16 bits as uint16) with row c divided by s16[c] in
+    one fp32 division; bf16 bits (uint16) when out_bf16, else fp32."""
+    P = as_f32(P)
+    if P.ndim == 1:
+        P = P.reshape(-1, 1)
+    R, C = P.shape
+    s16 = np.ascontiguousarray(s16, np.uint16)
+    if s16.shape[0] != R:
+        raise ValueError("s16 must have one entry per row of P")
+    out = np.empty((R, C), np.uint16 if out_bf16 else np.float32)
+    _load().orc_fold_scale(_p(P), R, C, _p(s16), 1 if out_bf16 else 0, _p(out))
+    return out

@@ -493,3 +493,199 @@ def test_apply_matches_dense_dequant():
     # and it approximates the unquantised layer
     yf = bf16_to_f32(x).astype(np.float64) @ bf16_to_f32(W).astype(np.float64).T
     assert np.linalg.norm(y - yf) < 0.2 * np.linalg.norm(yf)
+
+
+# ------------------------------------------------------------------ w_bit = 3
+def test_quant_group_w3_hand_case():
+    """3-bit symmetric: Delta = max / 3, codes in [-4, 3]; 3-bit asymmetric:
+    Delta = range / 7, z and codes in [0, 7] ([AWQ-guide] 三's 2^(w_bit-1) - 1
+    at w_bit = 3)."""
+    g = np.array([3.0, -1.5, 1.5, 0.5, -0.5, 2.5, -3.0] + [0.0] * 57, np.float32)
+    q, d, z = oracle.quant_group(g, oracle.SYM, w_bit=3)
+    assert d == np.float32(1.0) and z == 0
+    assert list(q[:7]) == [3, -2, 2, 0, 0, 2, -3]
+    g = np.array([5.0, -2.0, 0.5, 1.5, 2.5] + [0.0] * 59, np.float32)
+    q, d, z = oracle.quant_group(g, oracle.ASYM, w_bit=3)
+    assert d == np.float32(1.0) and z == 2                  # range 7 over 7 steps
+    assert list(q[:5]) == [7, 0, 2, 4, 4]                    # 0.5 -> 0, 1.5 -> 2, 2.5 -> 2 (+z)
+
+
+@pytest.mark.parametrize("qt", [0, 1])
+def test_quant_group_w3_enumeration(qt):
+    g = rng(80 + qt)
+    for trial in range(40):
+        w = (g.standard_normal(64) * 0.04).astype(np.float32)
+        for clip in (1.0, 0.8):
+            q, d, z = oracle.quant_group(w, qt, clip=clip, w_bit=3)
+            if qt == oracle.SYM:
+                a = np.float32(np.float64(np.abs(w).max()) * clip)
+                assert d == a / np.float32(3.0) and z == 0
+                lo, hi = -4, 3
+            else:
+                mxr = np.float32(np.float64(w.max()) * clip)
+                mnr = np.float32(np.float64(w.min()) * clip)
+                assert d == np.float32(mxr - mnr) / np.float32(7.0)
+                assert z == int(min(max(np.rint(np.float32(-mnr) / d), 0.0), 7.0))
+                lo, hi = -z, 7 - z
+            for k in range(64):
+                assert q[k] == _brute_nearest(float(np.float32(w[k]) / d), lo, hi) + z
+            if clip == 1.0:
+                err = np.abs(w.astype(np.float64) - (q - z) * float(d))
+                assert err.max() <= float(d) / 2 * (1 + 1e-6) + (float(d) if qt else 0.0)
+
+
+def test_search_w3_brute_force():
+    """The 3-bit search: losses equal brute-force losses over enumerated 3-bit
+    codes, and every 3-bit loss exceeds the 4-bit loss at the same alpha."""
+    O, I, N, gs = 3, 64, 8, 32
+    W, X = small_layer(O, I, N, wdtype="f32", xdtype="f32", seed=81, n_outliers=2)
+    sX = oracle.act_stats(X)
+    alpha = ALPHA_GRID[::6]
+    r3 = oracle.search_layer(W, X, sX, gs, oracle.SYM, alpha, w_bit=3)
+    r4 = oracle.search_layer(W, X, sX, gs, oracle.SYM, alpha, w_bit=4)
+    for k, a in enumerate(alpha):
+        s = oracle.scale_vector(sX, a)
+        Wf = oracle.as_f32(W)
+        c = np.zeros((O, I), np.int64)
+        d = np.zeros((O, I // gs), np.float32)
+        for o in range(O):
+            for j in range(I // gs):
+                wp = (Wf[o, j * gs:(j + 1) * gs] * s[j * gs:(j + 1) * gs]).astype(np.float32)
+                d[o, j] = np.float32(np.abs(wp).max()) / np.float32(3.0)
+                for t in range(gs):
+                    c[o, j * gs + t] = _brute_nearest(float(wp[t] / d[o, j]), -4, 3)
+        ref = _brute_loss_rows(W, X, s, gs, c, d, np.zeros((O, I // gs), np.int64)).sum() / (N * O)
+        assert r3["loss"][k] == pytest.approx(ref, rel=1e-12)
+        assert r3["loss"][k] > r4["loss"][k]
+
+
+# ------------------------------------------------------------------ joint grid
+def test_search_points_joint_grid_brute_force():
+    """Every (alpha, r) pair of a joint grid: the loss equals the brute-force
+    loss over enumerated codes at that pair; the best pair is the first
+    minimiser; pairs with r = 1 reproduce the alpha search."""
+    O, I, N, gs = 3, 64, 9, 32
+    W, X = small_layer(O, I, N, wdtype="f32", xdtype="f32", seed=82, n_outliers=2, outlier=25.0)
+    sX = oracle.act_stats(X)
+    al = ALPHA_GRID[::5]
+    cl = CLIP_GRID[::3]
+    A, C = np.meshgrid(al, cl, indexing="ij")
+    res = oracle.search_points(W, X, sX, gs, oracle.ASYM, A.ravel(), C.ravel())
+    ref = []
+    for a, r in zip(A.ravel(), C.ravel()):
+        s = oracle.scale_vector(sX, a)
+        c, d, z = _enum_quant_layer(W, s, gs, oracle.ASYM, float(r))
+        ref.append(_brute_loss_rows(W, X, s, gs, c, d, z).sum() / (N * O))
+    assert np.allclose(res["loss"], ref, rtol=1e-12)
+    assert res["best"] == int(np.argmin(ref))
+    plain = oracle.search_layer(W, X, sX, gs, oracle.ASYM, al)
+    assert np.array_equal(res["loss"].reshape(len(al), len(cl))[:, 0], plain["loss"])
+
+
+# ------------------------------------------------------------------ per-group clip
+def test_group_clip_brute_force():
+    """Per-group clip: each group's error at each ratio equals the brute-force
+    sum over tokens of its squared partial output error (codes by enumeration,
+    fsum over the group's columns); the chosen ratio is the first minimiser."""
+    O, I, N, gs = 2, 64, 6, 32
+    W, X = small_layer(O, I, N, wdtype="f32", xdtype="f32", seed=83, n_outliers=2, outlier=25.0)
+    sX = oracle.act_stats(X)
+    clip = CLIP_GRID[::2]
+    a = 0.4
+    for qt in (oracle.SYM, oracle.ASYM):
+        res = oracle.group_clip(W, X, sX, a, gs, qt, clip, want_err=True)
+        s = oracle.scale_vector(sX, a)
+        Wf, Xf = oracle.as_f32(W), oracle.as_f32(X)
+        for ri, r in enumerate(clip):
+            c, d, z = _enum_quant_layer(W, s, gs, qt, float(r))
+            for o in range(O):
+                for j in range(I // gs):
+                    cols = range(j * gs, (j + 1) * gs)
+                    dw = [(int(c[o, i]) - int(z[o, j])) * float(d[o, j]) / float(s[i]) - float(Wf[o, i])
+                          for i in cols]
+                    e = sum(math.fsum(float(Xf[n, i]) * dw[k] for k, i in enumerate(cols)) ** 2
+                            for n in range(N))
+                    assert res["err"][o, j, ri] == pytest.approx(e, rel=1e-12)
+        assert np.array_equal(res["best"], np.argmin(res["err"], axis=2))
+        assert np.all(np.min(res["err"], axis=2) <= res["err"][:, :, 0])
+
+
+def test_group_clip_single_ratio_and_pack():
+    """A one-point grid {1.0} selects index 0 everywhere; packing with per-group
+    ratios all equal to r equals packing at the layer ratio r; per-group
+    packing takes each group's codes at its own ratio."""
+    O, I, N, gs = 4, 256, 10, 64
+    W, X = small_layer(O, I, N, seed=84)
+    sX = oracle.act_stats(X)
+    res = oracle.group_clip(W, X, sX, 0.5, gs, oracle.ASYM, [1.0])
+    assert np.all(res["best"] == 0)
+    for qt in (oracle.SYM, oracle.ASYM):
+        flat = oracle.pack_int4(W, sX, 0.5, 0.85, gs, qt)
+        pg = oracle.pack_int4(W, sX, 0.5, 1.0, gs, qt, clip_g=np.full((O, I // gs), 0.85))
+        for k in ("qweight", "scales", "s16", "scales_f32"):
+            assert np.array_equal(flat[k], pg[k])
+        ratios = CLIP_GRID[rng(85).integers(0, len(CLIP_GRID), size=(O, I // gs))]
+        pg = oracle.pack_int4(W, sX, 0.5, 1.0, gs, qt, clip_g=ratios)
+        s = oracle.scale_vector(sX, 0.5)
+        nib = np.stack([(pg["qweight"] >> np.uint32(4 * k)) & np.uint32(15) for k in range(8)],
+                       axis=-1).reshape(O, I).astype(np.int64)
+        for o in range(O):
+            for j in range(I // gs):
+                c, d, z = _enum_quant_layer(W[o:o + 1], s, gs, qt, float(ratios[o, j]))
+                sl = slice(j * gs, (j + 1) * gs)
+                assert np.array_equal(nib[o, sl], c[0, sl] + (8 if qt == oracle.SYM else 0))
+                assert pg["scales_f32"][o, j] == d[0, j]
+
+
+# ------------------------------------------------------------------ fold of 1/s
+def test_apply_without_scale_is_integer_closed_form():
+    """s16 = None: x is used as is.  With Delta = 1 the result is x (codes - 8)^T
+    exactly, and equals the call with s16 = 1."""
+    r = rng(86)
+    M, I, O, gs = 2, 128, 5, 64
+    codes = r.integers(0, 16, size=(O, I)).astype(np.uint32)
+    qw = np.zeros((O, I // 8), np.uint32)
+    for k in range(8):
+        qw |= codes[:, k::8] << np.uint32(4 * k)
+    one16 = np.float16(1.0).view(np.uint16)
+    scales = np.full((O, I // gs), one16, np.uint16)
+    x = r.integers(-4, 5, size=(M, I)).astype(np.float32)
+    y = oracle.linear_w4a16(x, qw, scales, None, None, gs)
+    assert np.array_equal(y, (x.astype(np.int64) @ (codes.astype(np.int64) - 8).T).astype(np.float64))
+    y1 = oracle.linear_w4a16(x, qw, scales, None, np.full(I, one16, np.uint16), gs)
+    assert np.array_equal(y, y1)
+
+
+def test_fold_scale_closed_forms():
+    """Dividing by power-of-two scales is exact; s = 1 is the identity; random
+    scales round once in fp32 then to bf16 (checked against torch's own
+    float-to-bfloat16 conversion); a folded input through the apply without s
+    equals the unfolded input through the apply with s when the division is
+    exact."""
+    import torch
+    r = rng(87)
+    R, C = 64, 24
+    P = bf16_bits(r.standard_normal((R, C)).astype(np.float32))
+    k = r.integers(-6, 1, size=R)
+    s16 = (2.0 ** k).astype(np.float16).view(np.uint16)
+    out = oracle.fold_scale(P, s16)
+    assert np.array_equal(bf16_to_f32(out), bf16_to_f32(P) * (2.0 ** -k)[:, None].astype(np.float32))
+    ones = np.full(R, np.float16(1.0).view(np.uint16), np.uint16)
+    assert np.array_equal(oracle.fold_scale(P, ones), P)
+    s_r = r.uniform(0.01, 1.0, size=R).astype(np.float16)
+    got = oracle.fold_scale(P, s_r.view(np.uint16))
+    q32 = bf16_to_f32(P) / s_r.astype(np.float32)[:, None]      # one fp32 division
+    want = torch.from_numpy(q32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    got32 = oracle.fold_scale(P, s_r.view(np.uint16), out_bf16=False)
+    assert np.array_equal(got32, q32)
+    # fold then apply without s == apply with s, for exact (power-of-two) scales
+    I, O, gs = 64, 6, 32
+    W, X = small_layer(O, I, 12, seed=88)
+    sX = (2.0 ** r.integers(-5, 1, size=I)).astype(np.float32)
+    pk = oracle.pack_int4(W, sX, 1.0, 1.0, gs, oracle.ASYM)
+    x = bf16_bits(r.standard_normal((3, I)).astype(np.float32))
+    xf = oracle.fold_scale(x.T.copy(), pk["s16"]).T.copy()        # channel = row of P
+    y_fold = oracle.linear_w4a16(xf, pk["qweight"], pk["scales"], pk["zeros"], None, gs)
+    y = oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], gs)
+    assert np.array_equal(y_fold, y)
