@@ -1,27 +1,32 @@
 #!/usr/bin/env python
 """Benchmark of the AWQ per-layer scale search hot path on B200.
 
-One step = the whole path over one layer of the Llama-7B attention-projection
-workload (W 4096x4096 bf16, 4096 calibration tokens, symmetric INT4, group 128,
-20-point alpha grid): activation statistics -> fused grid search (fake
-quantisation, output-error contraction, loss reduction, argmin) -> INT4 packing
-at alpha* -> W4A16 apply at M = 1.
+One step = the whole path over one layer: activation statistics -> fused grid
+search (fake quantisation, output-error contraction, loss reduction, argmin)
+-> INT4 packing at alpha* -> W4A16 apply at M = 1.  The default layer is the
+Llama-13B up_proj at full calibration size: W 13824x5120 bf16, 65536
+calibration tokens (128 samples x 512), asymmetric INT4 with a uint4 zero
+point, group 128, 20-point alpha grid.  `--workload 2` runs the Llama-7B
+attention projection instead (4096x4096, 4096 tokens, symmetric).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 4|2]
 
 Metric: search TFLOP/s = grid * 2 * N * in * out per step / device time per
-step.  Inputs are resident in HBM when the timed region starts; three rotating
-copies of (W, X) (201 MB > 126 MB L2) keep each step's reads out of L2.  With N
-GPUs (torchrun, one process per GPU) every rank quantises its own layer
-(independent units, no data-path collective): weak scaling, time = max over
-ranks.  `--impl reference` times the CPU oracle on a bounded row sample of the
-same workload (rank 0 only).
+step.  Inputs are resident in HBM when the timed region starts.  On the
+default layer W (141.6 MB) and X (671.1 MB) are each larger than the 126 MB
+L2, so every step reads them from HBM; the 4096x4096 layer rotates three
+copies of (W, X) instead.  With N GPUs (torchrun, one process per GPU) every
+rank quantises its own layer (independent units, no data-path collective):
+weak scaling, time = max over ranks.  `--impl reference` times the CPU oracle
+on a bounded row sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -34,20 +39,28 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "AWQ search TFLOP/s (grid×2·N·in·out), ms/layer, % BF16 peak; W4A16 GB/s"
-WORKLOAD_ID = 2
-LAYER = "attn_proj"
 GROUP = 128
-ROTATE = 3
 APPLY_M = 1
+L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic of one search-kernel launch on this workload, from the ncu capture
-# summarised in profiles/search_kernel_attn_proj_4096x4096_n4096.md, valid only for the
-# kernel source it was taken on (sha256 of csrc/k_search.cu, first 16 hex).
+# Per benchmarked workload: the layer, its quantiser, how many (W, X) copies rotate
+# between steps, the default step count, and the rows of the oracle's timed sample.
+BENCH_WORKLOADS = {
+    4: {"layer": "up_proj", "quant": "asym", "rotate": 1, "steps": 10, "rows_per_core": 2},
+    2: {"layer": "attn_proj", "quant": "sym", "rotate": 3, "steps": 100, "rows_per_core": 48},
+}
+
 # Kernels of one step: statistics 2 (partial, final); search 9 (absmax, fp16 copy,
 # scale table 2, group parameters, search, row and block reductions, argmin);
 # packing 3 (scale table 2, pack); apply 1.
 LAUNCHES_PER_STEP = 15
-SEARCH_TRAFFIC = {"source_sha": "44d2be88c075101e", "bytes": 440555008}
+
+# DRAM bytes (read + write) of one search-kernel launch per workload, from an ncu
+# capture of that launch, valid only for the kernel source it was taken on
+# (sha256 of csrc/k_search.cu, first 16 hex digits).
+SEARCH_TRAFFIC = {
+    2: {"source_sha": "44d2be88c075101e", "bytes": 440555008},
+}
 
 
 def _env_int(k, d):
@@ -124,15 +137,24 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- our arm
-def bench_config(wl, world):
+def bench_config(wid, world):
     """The workload description both arms report (one layer per rank)."""
+    import synthetic
     from synthetic import ALPHA_GRID
-    L = wl.layers[0]
+    bw = BENCH_WORKLOADS[wid]
+    wl = synthetic.workload(wid)
+    L = next(l for l in wl.layers if l.name == bw["layer"])
     O, I, N = L.out, L.inp, wl.tokens
+    rot = bw["rotate"]
+    per_copy = 2 * (O * I + N * I)
+    if rot > 1:
+        l2 = f"{rot} rotating (W, X) copies, {rot * per_copy / 1e6:.0f} MB > 126 MB L2"
+    else:
+        l2 = (f"inputs larger than L2: W {2 * O * I / 1e6:.1f} MB and X {2 * N * I / 1e6:.1f} MB "
+              f"each > 126 MB, one copy")
     return {"workload": wl.name, "out": O, "in": I, "tokens": N, "grid": len(ALPHA_GRID),
-            "quant": "sym_int4", "group_size": GROUP, "apply_m": APPLY_M,
-            "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": f"{ROTATE} rotating (W, X) copies, {ROTATE * 2 * (O * I + N * I) / 1e6:.0f} MB > 126 MB L2"}
+            "quant": f"{bw['quant']}_int4", "group_size": GROUP, "apply_m": APPLY_M,
+            "parallelism": f"replicas{world}" if world > 1 else "single", "l2": l2}
 
 
 def max_over_ranks(value, world, device=None):
@@ -153,6 +175,12 @@ def job_tflops(flops_per_step, steps, world, ms):
     return flops_per_step * steps * world / (ms * 1e-3) / 1e12
 
 
+def _bf16_dev(a, dev):
+    import numpy as np
+    import torch
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -164,32 +192,32 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = synthetic.workload(WORKLOAD_ID)
-    L = wl.layers[0]
+    wid = args.workload
+    bw = BENCH_WORKLOADS[wid]
+    layer, quant, rot = bw["layer"], bw["quant"], bw["rotate"]
+    wl = synthetic.workload(wid)
+    L = next(l for l in wl.layers if l.name == layer)
     O, I, N, G = L.out, L.inp, wl.tokens, len(ALPHA_GRID)
     flops_step = G * 2.0 * N * I * O
 
-    def to_dev(a):
-        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
-
-    W_np = synthetic.layer_weights(WORKLOAD_ID, LAYER)
-    X_np = synthetic.layer_activations(WORKLOAD_ID, LAYER)
+    W_np = synthetic.layer_weights(wid, layer)
+    X_np = synthetic.layer_activations(wid, layer)
     x_np = synthetic.apply_activations(APPLY_M, I)
-    Ws = [to_dev(W_np) for _ in range(ROTATE)]
-    Xs = [to_dev(X_np) for _ in range(ROTATE)]
-    xd = to_dev(x_np)
+    Ws = [_bf16_dev(W_np, dev) for _ in range(rot)]
+    Xs = [_bf16_dev(X_np, dev) for _ in range(rot)]
+    xd = _bf16_dev(x_np, dev)
     alphas = [float(a) for a in ALPHA_GRID]
     awq.set_kernel_timing(True)
     search_ms = []
 
     def step(k, record):
-        Wd, Xd = Ws[k % ROTATE], Xs[k % ROTATE]
+        Wd, Xd = Ws[k % rot], Xs[k % rot]
         sX = awq.awq_act_stats(Xd)
-        res = awq.awq_search_layer(Wd, Xd, sX, GROUP, 4, "sym", alphas)
+        res = awq.awq_search_layer(Wd, Xd, sX, GROUP, 4, quant, alphas)
         if record:
             search_ms.append(awq.last_kernel_ms(awq.KT_SEARCH))
-        p = awq.awq_pack_int4(Wd, sX, alphas[res["best_alpha"]], 1.0, GROUP, "sym")
-        y = awq.awq_linear_w4a16(xd, p["qweight"], p["scales"], None, p["s16"], GROUP)
+        p = awq.awq_pack_int4(Wd, sX, alphas[res["best_alpha"]], 1.0, GROUP, quant)
+        y = awq.awq_linear_w4a16(xd, p["qweight"], p["scales"], p["zeros"], p["s16"], GROUP)
         return res, p, y
 
     for k in range(args.warmup):
@@ -225,14 +253,20 @@ def run_ours(args, rank, world, local_rank):
     x_h = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).pin_memory()
     qh = torch.empty(p["qweight"].shape, dtype=torch.int32).pin_memory()
     sh = torch.empty(p["scales"].shape, dtype=torch.float16).pin_memory()
+    zh = (torch.empty(p["zeros"].shape, dtype=torch.int32).pin_memory()
+          if p["zeros"] is not None else None)
     s16h = torch.empty(p["s16"].shape, dtype=torch.float16).pin_memory()
     yh = torch.empty(y.shape, dtype=torch.bfloat16).pin_memory()
     # Two device input buffers: step k+1's host-to-device copies run on a copy
     # stream while step k computes (a layer-by-layer quantiser loads the next
     # layer during the current one).  Every step still copies its own inputs.
+    del Ws, Xs
+    torch.cuda.empty_cache()
     comp_st = torch.cuda.current_stream()
     copy_st = torch.cuda.Stream()
-    bufs = [(torch.empty_like(Ws[0]), torch.empty_like(Xs[0]), torch.empty_like(xd)) for _ in range(2)]
+    bufs = [(torch.empty(W_h.shape, dtype=torch.bfloat16, device=dev),
+             torch.empty(X_h.shape, dtype=torch.bfloat16, device=dev),
+             torch.empty_like(xd)) for _ in range(2)]
     copied = [torch.cuda.Event() for _ in range(2)]
     done = [torch.cuda.Event() for _ in range(2)]
 
@@ -251,11 +285,13 @@ def run_ours(args, rank, world, local_rank):
         comp_st.wait_event(copied[b])
         Wd_e, Xd_e, xd_e = bufs[b]
         sX = awq.awq_act_stats(Xd_e)
-        r = awq.awq_search_layer(Wd_e, Xd_e, sX, GROUP, 4, "sym", alphas)
-        pk = awq.awq_pack_int4(Wd_e, sX, alphas[r["best_alpha"]], 1.0, GROUP, "sym")
-        yy = awq.awq_linear_w4a16(xd_e, pk["qweight"], pk["scales"], None, pk["s16"], GROUP)
+        r = awq.awq_search_layer(Wd_e, Xd_e, sX, GROUP, 4, quant, alphas)
+        pk = awq.awq_pack_int4(Wd_e, sX, alphas[r["best_alpha"]], 1.0, GROUP, quant)
+        yy = awq.awq_linear_w4a16(xd_e, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], GROUP)
         qh.copy_(pk["qweight"], non_blocking=True)
         sh.copy_(pk["scales"], non_blocking=True)
+        if zh is not None:
+            zh.copy_(pk["zeros"], non_blocking=True)
         s16h.copy_(pk["s16"], non_blocking=True)
         yh.copy_(yy, non_blocking=True)
         done[b].record(comp_st)
@@ -269,59 +305,56 @@ def run_ours(args, rank, world, local_rank):
                 issue_copy(k + 1)
             e2e_step(k)
 
-    e2e_run(max(2, args.warmup))
+    e2e_run(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(1, min(args.steps, 50))
+    e2e_steps = max(1, min(args.steps, 50 if wid == 2 else 5))
     e0.record()
     e2e_run(e2e_steps, e0)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     h2d = W_h.numel() * 2 + X_h.numel() * 2 + x_h.numel() * 2
-    d2h = qh.numel() * 4 + sh.numel() * 2 + s16h.numel() * 2 + yh.numel() * 2 + 8 * G + 4 * 8
+    d2h = (qh.numel() * 4 + sh.numel() * 2 + (zh.numel() * 4 if zh is not None else 0) +
+           s16h.numel() * 2 + yh.numel() * 2 + 8 * G + 4 * 8)
     e2e_value = job_tflops(flops_step, e2e_steps, world, e2e_ms)
+    del bufs
+    torch.cuda.empty_cache()
 
-    # ---- W4A16 apply at M = 1: rotating packed copies (> L2), one CUDA graph of launches.
-    n_copies = 16
-    packs = [awq.awq_pack_int4(Ws[0], sX_ := awq.awq_act_stats(Xs[0]), 0.5, 1.0, GROUP, "sym")
-             for _ in range(n_copies)]
+    # ---- W4A16 apply at M = 1 on this layer: rotating packed copies (> L2), one CUDA graph.
+    Wd0 = _bf16_dev(W_np, dev)
+    sX0 = awq.awq_act_stats(_bf16_dev(X_np[:4096], dev))
+    one = awq.awq_pack_int4(Wd0, sX0, 0.5, 1.0, GROUP, quant)
+    packed_bytes = sum(t.numel() * t.element_size() for t in
+                       (one["qweight"], one["scales"], one["s16"]) + ((one["zeros"],) if one["zeros"] is not None else ()))
+    n_copies = max(4, math.ceil(2 * L2_BYTES / packed_bytes))
+    packs = [one] + [awq.awq_pack_int4(Wd0, sX0, 0.5, 1.0, GROUP, quant) for _ in range(n_copies - 1)]
+    del Wd0
     ys = torch.empty((APPLY_M, O), dtype=torch.bfloat16, device=dev)
-    reps = 8
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
+    reps = max(1, 128 // n_copies)
     awq.set_kernel_timing(False)
-    with torch.cuda.stream(s):
+
+    def apply_all():
         for pk in packs:
-            awq.awq_linear_w4a16(xd, pk["qweight"], pk["scales"], None, pk["s16"], GROUP, out=ys)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for _ in range(reps):
-            for pk in packs:
-                awq.awq_linear_w4a16(xd, pk["qweight"], pk["scales"], None, pk["s16"], GROUP,
-                                     out=ys)
-    g.replay()
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    g.replay()
-    a1.record()
-    torch.cuda.synchronize()
-    apply_us = a0.elapsed_time(a1) * 1e3 / (reps * n_copies)
-    apply_bytes = O * I // 2 + O * (I // GROUP) * 2 + I * 2 + APPLY_M * I * 2 + APPLY_M * O * 2
-    del g
+            awq.awq_linear_w4a16(xd, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], GROUP,
+                                 out=ys)
+
+    apply_us = graph_time_us(apply_all, reps) / n_copies
+    apply_bytes = packed_bytes + APPLY_M * I * 2 + APPLY_M * O * 2
+    del packs
+    torch.cuda.empty_cache()
 
     block_apply = measure_block_apply(dev)
+    extra_search = measure_search_only(2, awq, dev) if wid != 2 else None
 
     pk_ = peaks()
     search_kernel_ms = statistics.mean(search_ms) if search_ms else None
     achieved = flops_step / (search_kernel_ms * 1e-3) / 1e12 if search_kernel_ms else None
     sha = source_sha(os.path.join(ROOT, "weight_only_quantization_awq_b200", "csrc", "k_search.cu"))
-    traffic = SEARCH_TRAFFIC["bytes"] if SEARCH_TRAFFIC["source_sha"] == sha else None
+    tr = SEARCH_TRAFFIC.get(wid)
+    traffic = tr["bytes"] if tr and tr["source_sha"] == sha else None
     out = {
         "metric": METRIC,
         "value": round(value, 3),
@@ -335,8 +368,9 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "f16",
         "data": "synthetic",
-        "config": bench_config(wl, world),
-        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms / e2e_steps, 4),
+        "config": bench_config(wid, world),
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s",
+                "ms_per_step": round(e2e_ms / e2e_steps, 4), "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
@@ -350,18 +384,78 @@ def run_ours(args, rank, world, local_rank):
                      "traffic": traffic},
         "ms_per_layer": round(ms_per_step, 4),
         "pct_bf16_peak": round(100.0 * value / world / pk_["bf16_tflops"], 2),
-        "w4a16": {"m": APPLY_M, "us_per_launch": round(apply_us, 3),
+        "w4a16": {"m": APPLY_M, "layer": f"{O}x{I}", "us_per_launch": round(apply_us, 3),
                   "gb_per_s": round(apply_bytes / (apply_us * 1e-6) / 1e9, 1),
                   "frac_hbm": round(apply_bytes / (apply_us * 1e-6) / 1e9 / pk_["hbm_gbs"], 4),
-                  "bytes": apply_bytes, "timing": f"CUDA graph of {reps * n_copies} launches over {n_copies} packed copies"},
+                  "bytes": apply_bytes,
+                  "timing": f"CUDA graph of {reps * n_copies} launches over {n_copies} packed copies"},
         "w4a16_block": {str(m): {**v, "frac_hbm": round(v["gb_per_s"] / pk_["hbm_gbs"], 4)}
                         for m, v in block_apply.items()},
     }
+    if extra_search is not None:
+        extra_search["frac"] = round(extra_search["tflops"] / pk_["bf16_tflops"], 4)
+        out["search_" + extra_search["workload"]] = extra_search
     if rank == 0 and world == 1:
-        out["cpu_baseline"] = cpu_baseline(W_np, X_np)
+        out["cpu_baseline"] = cpu_baseline(W_np, X_np, wid)
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     return out
+
+
+def graph_time_us(fn, reps):
+    """Device microseconds of one call of `fn` (a sequence of launches on the
+    current stream), from one CUDA graph that replays it `reps` times."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def measure_search_only(wid, awq, dev, reps=6):
+    """Search-kernel device time (library CUDA events) on another workload's
+    layer, rotating three input copies; reported beside the headline."""
+    import torch
+    import synthetic
+    from synthetic import ALPHA_GRID
+    bw = BENCH_WORKLOADS[wid]
+    wl = synthetic.workload(wid)
+    L = next(l for l in wl.layers if l.name == bw["layer"])
+    W_np = synthetic.layer_weights(wid, bw["layer"])
+    X_np = synthetic.layer_activations(wid, bw["layer"])
+    Ws = [_bf16_dev(W_np, dev) for _ in range(3)]
+    Xs = [_bf16_dev(X_np, dev) for _ in range(3)]
+    awq.set_kernel_timing(True)
+    alphas = [float(a) for a in ALPHA_GRID]
+    sXs = [awq.awq_act_stats(X) for X in Xs]
+    ms = []
+    for k in range(reps + 2):
+        awq.awq_search_layer(Ws[k % 3], Xs[k % 3], sXs[k % 3], GROUP, 4, bw["quant"], alphas)
+        if k >= 2:
+            ms.append(awq.last_kernel_ms(awq.KT_SEARCH))
+    awq.set_kernel_timing(False)
+    del Ws, Xs
+    torch.cuda.empty_cache()
+    flops = len(ALPHA_GRID) * 2.0 * wl.tokens * L.inp * L.out
+    kms = statistics.mean(ms)
+    return {"workload": wl.name, "kernel_ms": round(kms, 4),
+            "tflops": round(flops / (kms * 1e-3) / 1e12, 2), "algorithmic_flops": flops,
+            "timing": f"library CUDA events around the search kernel, mean of {reps} calls over 3 rotating input copies"}
 
 
 def measure_block_apply(dev, ms=(1, 16, 256), copies=2, reps=4):
@@ -389,37 +483,18 @@ def measure_block_apply(dev, ms=(1, 16, 256), copies=2, reps=4):
               for i in {i for _, _, i in BLOCK_LINEARS}}
         ys = [torch.empty((m, o), dtype=torch.bfloat16, device=dev) for _, o, _ in BLOCK_LINEARS]
 
-        def run_block(layer):
-            for k, (p, o, i) in enumerate(layer):
-                awq.awq_linear_w4a16(xs[i], p["qweight"], p["scales"], p["zeros"], p["s16"], GROUP,
-                                     out=ys[k])
-
-        s = torch.cuda.Stream()
-        s.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s):
+        def run_all():
             for layer in packs:
-                run_block(layer)
-        torch.cuda.current_stream().wait_stream(s)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(reps):
-                for layer in packs:
-                    run_block(layer)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        g.replay()
-        e1.record()
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+                for k, (p, o, i) in enumerate(layer):
+                    awq.awq_linear_w4a16(xs[i], p["qweight"], p["scales"], p["zeros"], p["s16"],
+                                         GROUP, out=ys[k])
+
+        us = graph_time_us(run_all, reps) / copies
         byts = sum(p["qweight"].numel() * 4 + p["scales"].numel() * 2 + p["zeros"].numel() * 4 +
                    p["s16"].numel() * 2 + m * i * 2 + m * o * 2 for p, o, i in packs[0])
         flops = sum(2.0 * m * o * i for _, o, i in BLOCK_LINEARS)
         out[m] = {"us_per_block": round(us, 2), "gb_per_s": round(byts / (us * 1e-6) / 1e9, 1),
                   "tflops": round(flops / (us * 1e-6) / 1e12, 2), "bytes": byts}
-        del g
     return out
 
 
@@ -430,28 +505,38 @@ def _oracle_threads():
     return int(os.environ["OMP_NUM_THREADS"])
 
 
-def oracle_step(W_np, X_np, rows):
+def oracle_step(W_np, X32, rows, qt):
     """The oracle's pass of the path on a row sample: statistics over all of X,
     the 20-point search evaluated on `rows`, packing of the whole layer."""
     import oracle
     from synthetic import ALPHA_GRID
-    sX = oracle.act_stats(X_np)
-    res = oracle.search_layer(W_np, X_np, sX, GROUP, 0, ALPHA_GRID, rows=rows)
-    oracle.pack_int4(W_np, sX, float(ALPHA_GRID[res["best_alpha"]]), 1.0, GROUP, 0)
+    sX = oracle.act_stats(X32)
+    res = oracle.search_layer(W_np, X32, sX, GROUP, qt, ALPHA_GRID, rows=rows)
+    oracle.pack_int4(W_np, sX, float(ALPHA_GRID[res["best_alpha"]]), 1.0, GROUP, qt)
     return res
 
 
-def cpu_baseline(W_np, X_np, rows_per_core=48):
+def _oracle_sample(wid, W_np, rows_scale=1.0):
     import numpy as np
     cores = _oracle_threads()
     O = W_np.shape[0]
-    R = min(O, rows_per_core * cores)
-    rows = np.arange(R, dtype=np.int64)
-    N, I = X_np.shape
+    R = min(O, max(1, int(BENCH_WORKLOADS[wid]["rows_per_core"] * cores * rows_scale)))
+    return cores, np.arange(R, dtype=np.int64)
+
+
+def cpu_baseline(W_np, X_np, wid):
+    import oracle
+    from synthetic import ALPHA_GRID
+    cores, rows = _oracle_sample(wid, W_np)
+    qt = 1 if BENCH_WORKLOADS[wid]["quant"] == "asym" else 0
+    X32 = oracle.as_f32(X_np)
+    O = W_np.shape[0]
+    N, I = X32.shape
+    R = rows.shape[0]
     t0 = time.perf_counter()
-    oracle_step(W_np, X_np, rows)
+    oracle_step(W_np, X32, rows, qt)
     dt = time.perf_counter() - t0
-    flops = 20 * 2.0 * N * I * R
+    flops = len(ALPHA_GRID) * 2.0 * N * I * R
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"full statistics and packing, 20-point search on the first {R} of {O} rows "
@@ -459,21 +544,24 @@ def cpu_baseline(W_np, X_np, rows_per_core=48):
 
 
 def run_reference(args):
-    import numpy as np
+    import oracle
     import synthetic
-    cores = _oracle_threads()
-    wl = synthetic.workload(WORKLOAD_ID)
-    L = wl.layers[0]
-    W_np = synthetic.layer_weights(WORKLOAD_ID, LAYER)
-    X_np = synthetic.layer_activations(WORKLOAD_ID, LAYER)
-    R = min(L.out, 4 * cores)
-    rows = np.arange(R, dtype=np.int64)
-    flops = 20 * 2.0 * wl.tokens * L.inp * R
+    from synthetic import ALPHA_GRID
+    wid = args.workload
+    bw = BENCH_WORKLOADS[wid]
+    qt = 1 if bw["quant"] == "asym" else 0
+    wl = synthetic.workload(wid)
+    L = next(l for l in wl.layers if l.name == bw["layer"])
+    W_np = synthetic.layer_weights(wid, bw["layer"])
+    X32 = oracle.as_f32(synthetic.layer_activations(wid, bw["layer"]))
+    cores, rows = _oracle_sample(wid, W_np, rows_scale=0.5)
+    R = rows.shape[0]
+    flops = len(ALPHA_GRID) * 2.0 * wl.tokens * L.inp * R
     for _ in range(args.warmup):
-        oracle_step(W_np, X_np, rows)
+        oracle_step(W_np, X32, rows, qt)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(W_np, X_np, rows)
+        oracle_step(W_np, X32, rows, qt)
     dt = time.perf_counter() - t0
     value = flops * args.steps / dt / 1e12
     sample = (f"per step: full statistics and packing, 20-point search on the first {R} of "
@@ -482,7 +570,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(dt * 1e3 / args.steps, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": bench_config(wl, 1),
+            "config": bench_config(wid, 1),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -492,10 +580,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, choices=sorted(BENCH_WORKLOADS), default=4)
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = BENCH_WORKLOADS[args.workload]["steps"]
     if args.warmup < 3:
         args.warmup = 3
     world = _env_int("WORLD_SIZE", 1)

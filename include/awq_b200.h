@@ -28,7 +28,8 @@
  *     and enqueues nothing.  A failing CUDA call returns AWQ_ERR_CUDA (see
  *     awq_last_error()).  In-kernel waits are bounded; a wait that gives up
  *     is reported as AWQ_ERR_TIMEOUT by the next synchronising entry point.
- *   - Supported: w_bit = 4; group_size in {32, 64, 128}; in % 64 == 0;
+ *   - Supported: w_bit in {3, 4} (3-bit codes are stored in the same 4-bit
+ *     container); group_size in {32, 64, 128}; in % 64 == 0;
  *     in % group_size == 0; any out >= 1 and N >= 1 (tails are masked).
  */
 #ifndef AWQ_B200_H
@@ -50,6 +51,9 @@ typedef enum {
 } awq_status_t;
 
 typedef enum { AWQ_F32 = 0, AWQ_BF16 = 1 } awq_dtype_t;
+
+/* Most (alpha, clip) points one awq_search_points call evaluates. */
+#define AWQ_MAX_POINTS 4096
 typedef enum { AWQ_SYM = 0, AWQ_ASYM = 1 } awq_quant_t;
 
 /* Library version, major*10000 + minor*100 + patch. */
@@ -70,7 +74,7 @@ const char *awq_last_error(void);
  * The mean accumulates in fp64: tokens are summed sequentially within chunks
  * of 128 consecutive tokens and the chunk partials are added in ascending
  * chunk order, then the fp64 mean is rounded once to fp32.
- * Requires in % 8 == 0.  Asynchronous.
+ * Requires in % 8 == 0 and N <= 2^40.  Asynchronous.
  */
 awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in,
                            float clamp_min, float *sX, void *stream);
@@ -89,6 +93,8 @@ awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in,
  * Quantizers: AWQ_SYM  Delta = max|w|/7, q = clamp(rint(w/Delta), -8, 7);
  *             AWQ_ASYM Delta = (max w - min w)/15, z = clamp(rint(-min/Delta), 0, 15),
  *                      q = clamp(rint(w/Delta) + z, 0, 15), value (q - z)*Delta.
+ *             At w_bit = 3: 3 and [-4, 3], 7 and [0, 7] ([AWQ-guide] 三's
+ *             2^(w_bit-1) - 1 at w_bit = 3).
  * W         : [out, in] device, fp32 or bf16 (w_dtype).
  * X         : [N, in] device, fp32 or bf16 (x_dtype).  The tensor-core
  *             contraction reads an fp16 copy of X scaled by one power of two
@@ -102,6 +108,10 @@ awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in,
  * loss_row  : optional [n_alpha + n_clip][out] fp32 device: per-row sums of
  *             squared output error (not divided by N).
  * best_alpha, best_clip : host, written (best_clip = -1 when n_clip == 0).
+ * The error term dW = Q(W*s)/s - W enters the fp16 contraction multiplied by
+ * one power of two per grid point (its bound over the layer lands in
+ * [2^14, 2^15)), undone exactly in the loss, so small weights keep fp16's
+ * full precision.
  * Synchronises `stream` (the losses are returned on the host).
  */
 awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t in,
@@ -111,6 +121,25 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
                               const double *clip, int n_clip,
                               double *loss, float *loss_row,
                               int *best_alpha, int *best_clip, void *stream);
+
+/*
+ * awq_search_points — the same loss at an arbitrary list of grid points:
+ * point k uses s = s_X^alpha[k] (normalised by its maximum) and clip ratio
+ * clip[k] ([AWQ-blog] Method: the scale search and the clipping of the enlarged
+ * weights, here searched jointly, e.g. every (alpha, r) pair of two grids,
+ * instead of r after alpha*).
+ * alpha, clip : [n_points] host, alpha in [0, 1], clip in (0, 1];
+ *               1 <= n_points <= AWQ_MAX_POINTS (evaluated 64 at a time).
+ * loss        : [n_points] host fp64, written.
+ * loss_row    : optional [n_points][out] fp32 device per-row sums.
+ * best        : host, the first k with the minimal loss.
+ * Other arguments as for awq_search_layer.  Synchronises `stream`.
+ */
+awq_status_t awq_search_points(const void *W, int w_dtype, int64_t out, int64_t in,
+                               const void *X, int x_dtype, int64_t N,
+                               const float *sX, int group_size, int w_bit, int quant,
+                               const double *alpha, const double *clip, int n_points,
+                               double *loss, float *loss_row, int *best, void *stream);
 
 /*
  * awq_pack_int4 — final quantisation at (alpha, clip) and INT4 packing
@@ -133,11 +162,53 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in,
                            uint16_t *s16, float *scales_f32, void *stream);
 
 /*
+ * awq_group_clip — one clip ratio per quantisation group ([AWQ-blog] Method,
+ * clipping of the enlarged weights, chosen group by group): with
+ * s = s_X^alpha (normalised by its maximum), for every output row o, group j
+ * and ratio clip_grid[r]:
+ *     err[o][j][r] = sum_n ( sum_{i in group j} X[n, i] * dW_r[o, i] )^2,
+ *     dW_r = Q_r(W*s)/s - W, Q_r the group quantiser with its bound(s) times r;
+ *     clip_idx[o][j] = the first r with the smallest err.
+ * The kernels reduce the tokens once into each group's Gram matrix
+ * H_j = X_j^T X_j (fp32 per 1024 tokens, fp64 across them) and evaluate
+ * err = dW_r^T H_j dW_r in fp32: exact in real arithmetic, so near-equal
+ * errors may order differently than a direct fp64 sum would.
+ * clip_grid : [n_clip] host, 1 <= n_clip <= 64, each in (0, 1].
+ * clip_idx  : [out][in/group_size] u8 device, written (for awq_pack_quant).
+ * err       : optional [out][in/group_size][n_clip] fp32 device, written.
+ * N <= 2^26.  Other arguments as for awq_search_layer.  Asynchronous.
+ */
+awq_status_t awq_group_clip(const void *W, int w_dtype, int64_t out, int64_t in,
+                            const void *X, int x_dtype, int64_t N, const float *sX,
+                            double alpha, int group_size, int w_bit, int quant,
+                            const double *clip_grid, int n_clip,
+                            uint8_t *clip_idx, float *err, void *stream);
+
+/*
+ * awq_pack_quant — awq_pack_int4 with the bit width and the clip choice open:
+ * w_bit in {3, 4} (3-bit codes in the same nibble layout: symmetric q + 8,
+ * asymmetric q), and either one ratio `clip` for the layer (clip_idx == NULL)
+ * or one ratio per quantisation group: clip_idx [out][in/group_size] u8
+ * device, each an index into clip_grid [n_clip] host (1 <= n_clip <= 64), as
+ * written by awq_group_clip ([AWQ-blog] Method, clipping of the enlarged
+ * weights, chosen per group).  Other arguments as for awq_pack_int4.
+ * Asynchronous.
+ */
+awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in,
+                            const float *sX, double alpha, double clip,
+                            const uint8_t *clip_idx, const double *clip_grid, int n_clip,
+                            int group_size, int w_bit, int quant,
+                            uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
+                            uint16_t *s16, float *scales_f32, void *stream);
+
+/*
  * awq_linear_w4a16 — the W4A16 layer that applies the result ([AWQ-guide] 三,
  * QuantLinear.forward: x rescaled by the per-channel scale, weight dequantised
  * per group, linear):
  *     y[m, o] = sum_i (x[m, i] / s16[i]) * (code[o, i] - z[o, i/gs]) * scales[o, i/gs]
  * with z = 8 when zeros == NULL (symmetric storage).  fp32 accumulation.
+ * s16 == NULL: x has already been divided by s (the division folded into the
+ * operator that produces x, see awq_fold_scale) and is used as is.
  * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.  in <= 49152.
  * Storage arguments as produced by awq_pack_int4.  Asynchronous.
  * Precision: x / s16 is rounded to fp16 after a power-of-two scale (2^-11
@@ -156,6 +227,33 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
                               int group_size, uint16_t *y, void *stream);
 
 /*
+ * awq_fold_scale — fold the division by s into the operator that produces
+ * this layer's input ([AWQ-blog] Method: X / s is merged into the preceding
+ * operator, so the W4A16 layer runs with s16 == NULL):
+ *     out[r][c] = P[r][c] / s16[r]    (one IEEE fp32 division; bf16: rounded
+ *                                      to nearest even)
+ * P    : [rows][cols] device, fp32 or bf16 (p_dtype): row r holds the producing
+ *        operator's parameters for channel r, e.g. an RMSNorm weight
+ *        (cols = 1) or a previous linear's weight rows (its output channels).
+ * s16  : [rows] fp16 bits device (awq_pack_int4's s16); must be nonzero.
+ * out  : [rows][cols] device, same dtype as P; may alias P (in place).
+ * Asynchronous.
+ */
+awq_status_t awq_fold_scale(const void *P, int p_dtype, int64_t rows, int64_t cols,
+                            const uint16_t *s16, void *out, void *stream);
+
+/*
+ * awq_wait_selftest — exercise the bounded in-kernel wait that guards every
+ * mbarrier wait of the search and apply kernels.  One CTA waits on an
+ * mbarrier that it arrives on only if `arrive` != 0, giving up after
+ * limit_cycles SM clock cycles (1 <= limit_cycles <= 4e9, about 2 s); no copy
+ * or MMA is in flight.  Returns AWQ_OK when the wait completed, AWQ_ERR_TIMEOUT
+ * when it gave up (reported through the same device error word as the search
+ * kernel).  Synchronises `stream`.
+ */
+awq_status_t awq_wait_selftest(int64_t limit_cycles, int arrive, void *stream);
+
+/*
  * awq_act_stats_noalloc — awq_act_stats without any device allocation.  The
  * AWQ pages have no counterpart: this exists for callers that cannot allocate
  * device memory when they compute the statistic (processes that hand nearly
@@ -165,7 +263,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
  * buffer compiled into the library instead of a temporary allocation, and
  * calls no allocating routine.
  * Limit: ceil(N / 128) * in <= 1,048,576; larger calls return
- * AWQ_ERR_UNSUPPORTED and enqueue nothing.
+ * AWQ_ERR_UNSUPPORTED and enqueue nothing.  Timed as kind 0 when timing is on.
  * The first call on a device looks up the buffer's device address (a
  * cudaGetSymbolAddress call); make that first call before any stream capture.
  * Every call shares the one buffer per device, so calls whose work overlaps on

@@ -53,7 +53,7 @@ def _search(**kw):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(W=NULL), ARG), (dict(wdt=7), ARG), (dict(out=0), ARG), (dict(quant=2), ARG),
-    (dict(gs=96), UNSUP), (dict(gs=256), UNSUP), (dict(inp=520), UNSUP), (dict(wbit=3), UNSUP),
+    (dict(gs=96), UNSUP), (dict(gs=256), UNSUP), (dict(inp=520), UNSUP), (dict(wbit=2), UNSUP), (dict(wbit=8), UNSUP),
     (dict(inp=576), UNSUP),          # a multiple of 64 that 128-column groups do not divide
     (dict(W=FAKE + 8), ALIGN), (dict(X=FAKE + 4), ALIGN), (dict(na=0), ARG), (dict(na=65), ARG),
     (dict(nc=-1), ARG), (dict(clip=NULL), ARG), (dict(N=0), ARG), (dict(loss=NULL), ARG),
@@ -108,3 +108,70 @@ def test_linear_rejects_on_host():
     assert call({2: 4160}) == UNSUP              # multiple of 64, not of the 128-column group
     assert call({8: 16}) == UNSUP
     assert call({0: FAKE + 2}) == ALIGN
+
+
+def test_search_points_rejects_on_host():
+    f = lib.awq_search_points
+    n = 6
+    a = (ctypes.c_double * n)(*([0.5] * n))
+    c = (ctypes.c_double * n)(*([1.0, 0.9] * 3))
+    loss = (ctypes.c_double * n)()
+    best = ctypes.c_int()
+    base = dict(W=FAKE, wdt=1, out=256, inp=512, X=FAKE, xdt=1, N=1024, sX=FAKE, gs=128, wbit=3,
+                quant=1, alpha=a, clip=c, n=n, loss=loss, lrow=NULL, best=ctypes.byref(best),
+                st=NULL)
+
+    def call(**kw):
+        args = dict(base)
+        args.update(kw)
+        return f(*args.values())
+    assert call(n=0) == ARG
+    assert call(n=4097) == ARG
+    assert call(clip=NULL) == ARG
+    assert call(alpha=(ctypes.c_double * n)(*([0.5] * 5 + [2.0]))) == ARG
+    assert call(clip=(ctypes.c_double * n)(*([1.0] * 5 + [0.0]))) == ARG
+    assert call(wbit=5) == UNSUP
+    assert call(gs=96) == UNSUP
+    assert call(best=NULL) == ARG
+    assert call(lrow=FAKE + 4) == ALIGN
+
+
+def test_pack_quant_rejects_on_host():
+    f = lib.awq_pack_quant
+    grid = (ctypes.c_double * 3)(1.0, 0.9, 0.8)
+    base = [FAKE, 1, 128, 256, FAKE, ctypes.c_double(0.5), ctypes.c_double(1.0), NULL, NULL, 0,
+            128, 3, 1, FAKE, FAKE, FAKE, FAKE, NULL, NULL]
+
+    def call(kw):
+        a = list(base)
+        for k, v in kw.items():
+            a[k] = v
+        return f(*a)
+    assert call({11: 2}) == UNSUP                # w_bit
+    assert call({7: FAKE}) == ARG                # per-group indices without a grid
+    assert call({7: FAKE, 8: grid, 9: 0}) == ARG
+    assert call({7: FAKE, 8: grid, 9: 65}) == ARG
+    assert call({7: FAKE, 8: (ctypes.c_double * 3)(1.0, 1.5, 0.8), 9: 3}) == ARG
+    assert call({15: NULL}) == ARG               # asymmetric without zeros
+    assert call({6: ctypes.c_double(0.0)}) == ARG
+
+
+def test_fold_and_selftest_reject_on_host():
+    f = lib.awq_fold_scale
+    assert f(NULL, 1, 16, 4, FAKE, FAKE, NULL) == ARG
+    assert f(FAKE, 2, 16, 4, FAKE, FAKE, NULL) == ARG
+    assert f(FAKE, 1, 0, 4, FAKE, FAKE, NULL) == ARG
+    assert f(FAKE, 1, 16, 4, NULL, FAKE, NULL) == ARG
+    assert f(FAKE + 1, 1, 16, 4, FAKE, FAKE, NULL) == ALIGN
+    assert f(FAKE + 2, 0, 16, 4, FAKE, FAKE, NULL) == ALIGN
+    g = lib.awq_wait_selftest
+    assert g(0, 0, NULL) == ARG
+    assert g(5_000_000_000, 0, NULL) == ARG
+
+
+def test_linear_accepts_missing_scale_vector_on_host():
+    """s16 = NULL (x already divided by s) passes validation: the call only fails
+    later, for want of a device, not as an argument error."""
+    f = lib.awq_linear_w4a16
+    st = f(FAKE, 1, 4096, 4096, FAKE, FAKE, NULL, NULL, 128, FAKE, NULL)
+    assert st not in (ARG, ALIGN, UNSUP)

@@ -53,7 +53,8 @@ def test_single_rank_is_identity():
 
 def test_reference_arm_other_ranks_exit_silently():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1"],
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--workload", "2"],
                        env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
@@ -67,7 +68,7 @@ def test_reference_arm_line_on_rank0():
     import synthetic
     env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0", OMP_NUM_THREADS="4")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "0"],
+                        "--steps", "1", "--warmup", "0", "--workload", "2"],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [l for l in r.stdout.splitlines() if l.strip()]
@@ -79,7 +80,8 @@ def test_reference_arm_line_on_rank0():
         assert k in d, k
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["value"] > 0 and d["steps"] == 1
-    assert d["config"] == bench.bench_config(synthetic.workload(bench.WORKLOAD_ID), 1)
+    assert d["config"] == bench.bench_config(2, 1)
+    assert d["config"]["workload"] == synthetic.workload(2).name
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     cb = d["cpu_baseline"]

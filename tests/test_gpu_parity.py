@@ -230,14 +230,19 @@ def test_linear_w4a16_parity(awq, M, O, I, gs, qt):
 
 
 @pytest.mark.parametrize("M", [1, 16, 256])
-def test_linear_w4a16_block_shape(awq, M):
-    """A 4096x4096 linear of the decoder block, packed by the GPU itself."""
-    W = synthetic.layer_weights(5, "o")
-    X = synthetic.layer_activations(5, "o", tokens=512)
+@pytest.mark.parametrize("layer", ["o", "gate", "down"])
+def test_linear_w4a16_block_shape(awq, M, layer):
+    """The decoder block's linear shapes (o 4096x4096, gate 11008x4096, down
+    4096x11008), packed by the GPU itself."""
+    src = {"o": "o", "gate": "gate_up", "down": "down"}[layer]
+    W = synthetic.layer_weights(5, src)
+    if layer == "gate":
+        W = np.ascontiguousarray(W[:11008])
+    X = synthetic.layer_activations(5, src, tokens=512)
     Wd = dev(W)
     sXd = awq.awq_act_stats(dev(X))
     p = awq.awq_pack_int4(Wd, sXd, 0.5, 1.0, 128, 1)
-    x = apply_activations(M, 4096)
+    x = apply_activations(M, W.shape[1])
     y = awq.awq_linear_w4a16(dev(x), p["qweight"], p["scales"], p["zeros"], p["s16"], 128)
     y_ref = oracle.linear_w4a16(x, u32(p["qweight"]), u16(p["scales"]), u32(p["zeros"]),
                                 u16(p["s16"]), 128)

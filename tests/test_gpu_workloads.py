@@ -109,7 +109,7 @@ def test_workload4_up_proj_asym(awq):
     check_codes(awq, W, Wd, sXd, float(ALPHA_GRID[got["best_alpha"]]), 1.0, 1)
 
 
-@pytest.mark.parametrize("layer", ["o", "down"])
+@pytest.mark.parametrize("layer", ["o", "down", "qkv", "gate_up"])
 def test_workload5_asym_with_clip(awq, layer):
     W, X, Wd, Xd, sXd, sX, got, lr, rows = run_layer(awq, 5, layer, 1, 6, clip=CLIP_GRID,
                                                      seed=51)

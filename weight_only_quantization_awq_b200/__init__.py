@@ -8,8 +8,12 @@ names:
     awq_act_stats(X)                         -> s_X = mean |X| per input channel
     awq_act_stats_noalloc(X)                 -> the same without any device allocation
     awq_search_layer(W, X, sX, ...)          -> losses over the alpha (and clip) grid, argmin
+    awq_search_points(W, X, sX, alpha, clip) -> losses at listed (alpha, clip) points, argmin
     awq_pack_int4(W, sX, alpha, clip, ...)   -> packed INT4 codes, fp16 scales, zeros, s
-    awq_linear_w4a16(x, packed...)           -> y = (x / s) @ dequant(W)^T
+    awq_pack_quant(W, sX, alpha, ...)        -> the same at w_bit 3 or 4, per-group clip ratios
+    awq_linear_w4a16(x, packed...)           -> y = (x / s) @ dequant(W)^T (s16=None: x pre-divided)
+    awq_fold_scale(P, s16)                   -> P / s per row (1/s folded into the previous op)
+    awq_wait_selftest(limit, arrive)         -> status of one bounded in-kernel wait
 
 Importing raises ImportError when the compiled library is missing; there is no
 fallback implementation.
@@ -61,6 +65,16 @@ def _load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.awq_linear_w4a16.argtypes = [P, L, L, L, P, P, P, P, I, P, P]
     lib.awq_act_stats_noalloc.restype = I
     lib.awq_act_stats_noalloc.argtypes = [P, I, L, L, F, P, P]
+    lib.awq_search_points.restype = I
+    lib.awq_search_points.argtypes = [P, I, L, L, P, I, L, P, I, I, I, P, P, I, P, P, P, P]
+    lib.awq_pack_quant.restype = I
+    lib.awq_pack_quant.argtypes = [P, I, L, L, P, D, D, P, P, I, I, I, I, P, P, P, P, P, P]
+    lib.awq_group_clip.restype = I
+    lib.awq_group_clip.argtypes = [P, I, L, L, P, I, L, P, D, I, I, I, P, I, P, P, P]
+    lib.awq_fold_scale.restype = I
+    lib.awq_fold_scale.argtypes = [P, I, L, L, P, P, P]
+    lib.awq_wait_selftest.restype = I
+    lib.awq_wait_selftest.argtypes = [L, I, P]
     lib.awq_set_kernel_timing.restype = None
     lib.awq_set_kernel_timing.argtypes = [I]
     lib.awq_last_kernel_ms.restype = D
@@ -71,8 +85,12 @@ def _load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 lib = _load_library()
 
 EXPORTS = ("awq_version", "awq_status_string", "awq_last_error", "awq_act_stats",
-           "awq_search_layer", "awq_pack_int4", "awq_linear_w4a16", "awq_set_kernel_timing",
+           "awq_search_layer", "awq_search_points", "awq_group_clip", "awq_pack_int4",
+           "awq_pack_quant",
+           "awq_linear_w4a16", "awq_fold_scale", "awq_wait_selftest", "awq_set_kernel_timing",
            "awq_last_kernel_ms", "awq_act_stats_noalloc")
+
+MAX_POINTS = 4096
 
 KT_STATS, KT_SEARCH, KT_PACK, KT_APPLY = 0, 1, 2, 3
 
@@ -121,12 +139,26 @@ def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
     return t
 
 
+def _out(t: torch.Tensor, name: str, like: torch.Tensor, dtype: torch.dtype, numel: int):
+    """A caller-supplied result tensor: CUDA, contiguous, on `like`'s device, of
+    `dtype` and `numel` elements (the library writes exactly that many)."""
+    _dev(t, name)
+    if t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, the inputs on {like.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+    return t
+
+
 def awq_act_stats(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.Tensor | None = None):
     """s_X[i] = max(clamp_min, mean_n |X[n, i]|) for X [N, in] (fp32 or bf16)."""
     _dev(X, "X")
     N, inp = X.shape
     if out is None:
         out = torch.empty(inp, dtype=torch.float32, device=X.device)
+    _out(out, "out", X, torch.float32, inp)
     _check("awq_act_stats", lib.awq_act_stats(X.data_ptr(), _dtype_code(X), N, inp,
                                               float(clamp_min), out.data_ptr(), _stream(X)))
     return out
@@ -140,6 +172,7 @@ def awq_act_stats_noalloc(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.T
     N, inp = X.shape
     if out is None:
         out = torch.empty(inp, dtype=torch.float32, device=X.device)
+    _out(out, "out", X, torch.float32, inp)
     _check("awq_act_stats_noalloc",
            lib.awq_act_stats_noalloc(X.data_ptr(), _dtype_code(X), N, inp, float(clamp_min),
                                      out.data_ptr(), _stream(X)))
@@ -171,6 +204,113 @@ def awq_search_layer(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, group_s
     return {"loss": loss, "loss_row": lr, "best_alpha": ba.value, "best_clip": bc.value}
 
 
+def awq_search_points(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, alpha, clip,
+                      group_size: int = 128, w_bit: int = 4, quant="sym", loss_row: bool = False):
+    """The loss at each listed (alpha[k], clip[k]) point (a joint grid).  Returns
+    dict(loss: np.ndarray [n] fp64, loss_row: tensor [n, out] fp32 or None, best)."""
+    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
+    out_f, inp = W.shape
+    N = X.shape[0]
+    if X.shape[1] != inp or sX.numel() != inp:
+        raise ValueError("W, X and sX disagree on the input width")
+    a = np.ascontiguousarray(np.asarray(alpha, dtype=np.float64).ravel())
+    c = np.ascontiguousarray(np.asarray(clip, dtype=np.float64).ravel())
+    if a.size != c.size:
+        raise ValueError("alpha and clip must list the same number of points")
+    loss = np.empty(a.size, np.float64)
+    lr = (torch.empty((a.size, out_f), dtype=torch.float32, device=W.device)
+          if loss_row else None)
+    best = ctypes.c_int()
+    st = lib.awq_search_points(
+        W.data_ptr(), _dtype_code(W), out_f, inp, X.data_ptr(), _dtype_code(X), N, sX.data_ptr(),
+        group_size, w_bit, _quant_code(quant), a.ctypes.data, c.ctypes.data, a.size,
+        loss.ctypes.data, lr.data_ptr() if lr is not None else None, ctypes.byref(best), _stream(W))
+    _check("awq_search_points", st)
+    return {"loss": loss, "loss_row": lr, "best": best.value}
+
+
+def awq_group_clip(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, alpha: float, clip_grid,
+                   group_size: int = 128, w_bit: int = 4, quant="asym", want_err: bool = False):
+    """One clip ratio per (row, group) at s = s_X^alpha: the first ratio of
+    clip_grid minimising the group's own output error.  Returns dict(clip_idx:
+    uint8 [out, in/gs] device, err: fp32 [out, in/gs, n_clip] device or None)."""
+    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
+    out_f, inp = W.shape
+    N = X.shape[0]
+    if X.shape[1] != inp or sX.numel() != inp:
+        raise ValueError("W, X and sX disagree on the input width")
+    g = np.ascontiguousarray(np.asarray(clip_grid, dtype=np.float64).ravel())
+    nG = inp // group_size
+    idx = torch.empty((out_f, nG), dtype=torch.uint8, device=W.device)
+    err = (torch.empty((out_f, nG, g.size), dtype=torch.float32, device=W.device)
+           if want_err else None)
+    st = lib.awq_group_clip(
+        W.data_ptr(), _dtype_code(W), out_f, inp, X.data_ptr(), _dtype_code(X), N, sX.data_ptr(),
+        float(alpha), group_size, w_bit, _quant_code(quant), g.ctypes.data, g.size, idx.data_ptr(),
+        err.data_ptr() if err is not None else None, _stream(W))
+    _check("awq_group_clip", st)
+    return {"clip_idx": idx, "err": err}
+
+
+def awq_pack_quant(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float = 1.0,
+                   group_size: int = 128, quant="sym", w_bit: int = 4,
+                   clip_idx: torch.Tensor | None = None, clip_grid=None,
+                   scales_f32: bool = False):
+    """Packed storage at w_bit 3 or 4, with one clip ratio for the layer or, given
+    clip_idx (uint8 [out, in/gs] device) and clip_grid, one per group.  Same
+    dict as awq_pack_int4."""
+    _dev(W, "W"), _dev(sX, "sX")
+    out_f, inp = W.shape
+    q = _quant_code(quant)
+    nG = inp // group_size
+    dev = W.device
+    grid = None
+    if clip_idx is not None:
+        _out(clip_idx, "clip_idx", W, torch.uint8, out_f * nG)
+        grid = np.ascontiguousarray(np.asarray(clip_grid, dtype=np.float64).ravel())
+    qweight = torch.empty((out_f, inp // 8), dtype=torch.int32, device=dev)
+    scales = torch.empty((out_f, nG), dtype=torch.float16, device=dev)
+    zeros = (torch.empty((out_f, (nG + 7) // 8), dtype=torch.int32, device=dev)
+             if q == AWQ_ASYM else None)
+    s16 = torch.empty(inp, dtype=torch.float16, device=dev)
+    sf = torch.empty((out_f, nG), dtype=torch.float32, device=dev) if scales_f32 else None
+    st = lib.awq_pack_quant(
+        W.data_ptr(), _dtype_code(W), out_f, inp, sX.data_ptr(), float(alpha), float(clip),
+        clip_idx.data_ptr() if clip_idx is not None else None,
+        grid.ctypes.data if grid is not None else None, grid.size if grid is not None else 0,
+        group_size, w_bit, q, qweight.data_ptr(), scales.data_ptr(),
+        zeros.data_ptr() if zeros is not None else None, s16.data_ptr(),
+        sf.data_ptr() if sf is not None else None, _stream(W))
+    _check("awq_pack_quant", st)
+    return {"qweight": qweight, "scales": scales, "zeros": zeros, "s16": s16, "scales_f32": sf,
+            "group_size": group_size}
+
+
+def awq_fold_scale(P: torch.Tensor, s16: torch.Tensor, out: torch.Tensor | None = None):
+    """P [rows, cols] (or [rows]) fp32 / bf16 with row r divided by s16[r]: the
+    division of the next layer's input by s folded into the operator that
+    produces it (an RMSNorm weight, a previous linear's weight rows)."""
+    _dev(P, "P"), _dev(s16, "s16")
+    rows = P.shape[0]
+    cols = P.numel() // rows if rows else 0
+    if s16.numel() != rows or s16.dtype != torch.float16:
+        raise ValueError("s16 must be fp16 with one entry per row of P")
+    if out is None:
+        out = torch.empty_like(P)
+    _out(out, "out", P, P.dtype, P.numel())
+    _check("awq_fold_scale", lib.awq_fold_scale(P.data_ptr(), _dtype_code(P), rows, cols,
+                                                s16.data_ptr(), out.data_ptr(), _stream(P)))
+    return out
+
+
+def awq_wait_selftest(limit_cycles: int, arrive: bool, device=None) -> int:
+    """Run the bounded-wait self-test on the current stream; returns the status
+    code (0 = the wait completed, 5 = AWQ_ERR_TIMEOUT) instead of raising."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    st = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    return int(lib.awq_wait_selftest(int(limit_cycles), 1 if arrive else 0, st))
+
+
 def awq_pack_int4(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float = 1.0,
                   group_size: int = 128, quant="sym", scales_f32: bool = False):
     """Packed storage at (alpha, clip): dict(qweight int32 [out, in/8] (u32 bits),
@@ -198,19 +338,23 @@ def awq_pack_int4(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float =
 
 
 def awq_linear_w4a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
-                     zeros: torch.Tensor | None, s16: torch.Tensor, group_size: int = 128,
+                     zeros: torch.Tensor | None, s16: torch.Tensor | None, group_size: int = 128,
                      out: torch.Tensor | None = None):
-    """y [M, out] bf16 = (x / s16) @ dequant(qweight, scales, zeros)^T for bf16 x [M, in]."""
-    _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales"), _dev(s16, "s16")
+    """y [M, out] bf16 = (x / s16) @ dequant(qweight, scales, zeros)^T for bf16 x [M, in];
+    s16=None when x has already been divided by s (awq_fold_scale)."""
+    _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales")
+    if s16 is not None:
+        _dev(s16, "s16")
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bfloat16")
     M, inp = x.shape
     out_f = qweight.shape[0]
     if out is None:
         out = torch.empty((M, out_f), dtype=torch.bfloat16, device=x.device)
+    _out(out, "out", x, torch.bfloat16, M * out_f)
     st = lib.awq_linear_w4a16(
         x.data_ptr(), M, inp, out_f, qweight.data_ptr(), scales.data_ptr(),
-        zeros.data_ptr() if zeros is not None else None, s16.data_ptr(), group_size,
-        out.data_ptr(), _stream(x))
+        zeros.data_ptr() if zeros is not None else None,
+        s16.data_ptr() if s16 is not None else None, group_size, out.data_ptr(), _stream(x))
     _check("awq_linear_w4a16", st)
     return out

@@ -167,15 +167,16 @@ bool valid_dtype(int d) { return d == AWQ_F32 || d == AWQ_BF16; }
 // Optional CUDA-event timing of the main kernels (see awq_set_kernel_timing).
 constexpr int KT_KINDS = 4;
 thread_local bool t_timing = false;
+constexpr int KT_MAX = 64;          // launches one entry point may bracket
 struct KTimer {
-    cudaEvent_t beg[2] = {nullptr, nullptr}, end[2] = {nullptr, nullptr};
+    cudaEvent_t beg[KT_MAX] = {}, end[KT_MAX] = {};
     int n = 0;
 };
 thread_local KTimer t_kt[KT_KINDS];
 
-void kt_reset(int kind) {
+void kt_reset_impl(int kind) {
     KTimer &k = t_kt[kind];
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < KT_MAX; ++i) {
         if (k.beg[i]) cudaEventDestroy(k.beg[i]);
         if (k.end[i]) cudaEventDestroy(k.end[i]);
         k.beg[i] = k.end[i] = nullptr;
@@ -183,19 +184,19 @@ void kt_reset(int kind) {
     k.n = 0;
 }
 
-void kt_begin(int kind, cudaStream_t st) {
+void kt_begin_impl(int kind, cudaStream_t st) {
     if (!t_timing) return;
     KTimer &k = t_kt[kind];
-    if (k.n >= 2) return;
+    if (k.n >= KT_MAX) return;
     cudaEventCreate(&k.beg[k.n]);
     cudaEventCreate(&k.end[k.n]);
     cudaEventRecord(k.beg[k.n], st);
 }
 
-void kt_end(int kind, cudaStream_t st) {
+void kt_end_impl(int kind, cudaStream_t st) {
     if (!t_timing) return;
     KTimer &k = t_kt[kind];
-    if (k.n >= 2 || !k.end[k.n]) return;
+    if (k.n >= KT_MAX || !k.end[k.n]) return;
     cudaEventRecord(k.end[k.n], st);
     ++k.n;
 }
@@ -219,10 +220,17 @@ awq_status_t check_layer(const void *W, int w_dtype, int64_t out, int64_t in, in
 }  // namespace
 
 void awq::set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
+void awq::kt_reset(int kind) { kt_reset_impl(kind); }
+void awq::kt_begin(int kind, cudaStream_t st) { kt_begin_impl(kind, st); }
+void awq::kt_end(int kind, cudaStream_t st) { kt_end_impl(kind, st); }
+
+using awq::kt_begin;
+using awq::kt_end;
+using awq::kt_reset;
 
 extern "C" {
 
-int awq_version(void) { return 100; }
+int awq_version(void) { return 200; }
 
 const char *awq_status_string(int status) {
     switch (status) {
@@ -240,7 +248,7 @@ const char *awq_last_error(void) { return g_last_error.c_str(); }
 
 void awq_set_kernel_timing(int enable) {
     t_timing = enable != 0;
-    for (int k = 0; k < KT_KINDS; ++k) kt_reset(k);
+    for (int k = 0; k < KT_KINDS; ++k) kt_reset_impl(k);
 }
 
 double awq_last_kernel_ms(int kind) {
@@ -264,7 +272,7 @@ awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in, fl
     if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
     if (N < 1 || in < 1) return fail(AWQ_ERR_ARG, "bad shape N=%lld in=%lld", (long long)N, (long long)in);
     if (in % 8 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of 8", (long long)in);
-    if (N > (int64_t(1) << 31) / 1) return fail(AWQ_ERR_UNSUPPORTED, "N too large");
+    if (N > (int64_t(1) << 40)) return fail(AWQ_ERR_UNSUPPORTED, "N above 2^40");
     if (!(clamp_min >= 0.0f)) return fail(AWQ_ERR_ARG, "clamp_min must be >= 0");
     if (!aligned16(X) || !aligned16(sX)) return fail(AWQ_ERR_ALIGN, "X/sX not 16-byte aligned");
     int sms;
@@ -282,18 +290,123 @@ awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in, fl
     return AWQ_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Device buffers of one search call, shared by its phases (each phase evaluates
+// at most MAX_GRID grid points).
+struct SearchBufs {
+    uint16_t *x16;
+    float *sn;
+    char *sc_scratch;
+    float4 *qparam;
+    float *part;
+    double *blocksum;
+    int *flags;          // [0] best alpha, [1] best clip, [2] device error word, [3] max|X| bits, [4] X exponent
+    unsigned *dw_bits;
+    int *dw_exp;
+};
+
+awq_status_t reserve_search(Workspace &ws, SearchBufs *b, int64_t out, int64_t in, int64_t N,
+                            int gs, int Gmax, int n_loss, double **loss_d) {
+    const int64_t nG = in / gs;
+    const int64_t TB = (N + awq::TILE_N - 1) / awq::TILE_N;
+    size_t bytes = 0;
+    bytes += Workspace::up(sizeof(uint16_t) * N * in);
+    bytes += Workspace::up(sizeof(float) * 2 * Gmax * in);
+    bytes += Workspace::up(awq::scale_scratch_bytes(Gmax, in));
+    bytes += Workspace::up(sizeof(float4) * Gmax * out * nG);
+    bytes += Workspace::up(sizeof(float) * Gmax * TB * out);
+    bytes += Workspace::up(sizeof(double) * n_loss);
+    bytes += Workspace::up(sizeof(double) * awq::reduce_scratch_doubles(Gmax, out));
+    bytes += Workspace::up(sizeof(int) * 8);
+    bytes += Workspace::up(sizeof(unsigned) * Gmax);
+    bytes += Workspace::up(sizeof(int) * Gmax);
+    if (awq_status_t s = ws.reserve(bytes)) return s;
+    b->x16 = ws.take<uint16_t>(N * in);
+    b->sn = ws.take<float>(2 * Gmax * in);
+    b->sc_scratch = ws.take<char>(awq::scale_scratch_bytes(Gmax, in));
+    b->qparam = ws.take<float4>(Gmax * out * nG);
+    b->part = ws.take<float>(Gmax * TB * out);
+    *loss_d = ws.take<double>(n_loss);
+    b->blocksum = ws.take<double>(awq::reduce_scratch_doubles(Gmax, out));
+    b->flags = ws.take<int>(8);
+    b->dw_bits = ws.take<unsigned>(Gmax);
+    b->dw_exp = ws.take<int>(Gmax);
+    return AWQ_OK;
+}
+
+// One phase of the search: G <= MAX_GRID grid points, point g at
+// alpha.value[g] (or alpha.value[*best_idx] for all g when best_idx is given)
+// and clip ratio clip.value[g]; the losses go to loss_d[0..G) (device) and the
+// optional per-row sums to loss_row[g][out].
+awq_status_t search_phase(const SearchBufs &b, const void *W, bool w_bf16, int64_t out, int64_t in,
+                          int64_t N, const float *sX, int gs, int wbit, bool asym,
+                          const awq::GridParams &alpha, const int *best_idx,
+                          const awq::GridParams &clip, int G, double *loss_d, float *loss_row,
+                          int sms, cudaStream_t st) {
+    const int64_t TB = (N + awq::TILE_N - 1) / awq::TILE_N;
+    bool clipped = false;
+    for (int g = 0; g < G; ++g) clipped |= clip.value[g] != 1.0;
+    AWQ_CUDA(awq::launch_scale_table(sX, in, alpha, G, best_idx, b.sn, b.sc_scratch, st));
+    AWQ_CUDA(awq::launch_group_params(W, w_bf16, out, in, gs, asym, wbit, b.sn, clip, G, b.qparam,
+                                      b.dw_bits, b.dw_exp, st));
+    awq::SearchArgs a{};
+    a.w_bf16 = w_bf16;
+    a.O = out;
+    a.I = in;
+    a.N = N;
+    a.gs = gs;
+    a.G = G;
+    a.clamp = asym || clipped;
+    a.part = b.part;
+    a.err = b.flags + 2;
+    a.wait = awq::AWQ_DEFAULT_WAIT_CYCLES;
+    awq::SearchMaps maps;
+    if (awq_status_t s = make_search_maps(&maps, b.x16, N, W, w_bf16, out, in, b.sn, b.qparam, G, gs))
+        return s;
+    kt_begin(1, st);
+    AWQ_CUDA(awq::launch_search(a, maps, sms, st));
+    kt_end(1, st);
+    AWQ_CUDA(awq::launch_reduce_loss(b.part, G, TB, out, N, b.flags + 4, b.dw_exp, loss_d, loss_row,
+                                     b.blocksum, st));
+    return AWQ_OK;
+}
+
+awq_status_t device_error(int word, const char *what) {
+    if (word != 0)
+        return fail(AWQ_ERR_TIMEOUT, "%s: a bounded wait gave up (device error %d)", what, word);
+    return AWQ_OK;
+}
+
+awq_status_t check_search_inputs(const void *W, int w_dtype, int64_t out, int64_t in, const void *X,
+                                 int x_dtype, int64_t N, const float *sX, int group_size, int w_bit,
+                                 int quant, const float *loss_row) {
+    if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
+    if (w_bit != 3 && w_bit != 4) return fail(AWQ_ERR_UNSUPPORTED, "w_bit %d (3 or 4)", w_bit);
+    if (!X || !sX) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
+    if (N < 1 || N > (int64_t(1) << 30)) return fail(AWQ_ERR_ARG, "bad N=%lld", (long long)N);
+    if (!aligned16(X) || !aligned16(sX) || (loss_row && !aligned16(loss_row)))
+        return fail(AWQ_ERR_ALIGN, "device pointer not 16-byte aligned");
+    return AWQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t in, const void *X,
                               int x_dtype, int64_t N, const float *sX, int group_size, int w_bit,
                               int quant, const double *alpha, int n_alpha, const double *clip,
                               int n_clip, double *loss, float *loss_row, int *best_alpha,
                               int *best_clip, void *stream) {
     g_last_error.clear();
-    if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
-    if (w_bit != 4) return fail(AWQ_ERR_UNSUPPORTED, "w_bit %d (only 4)", w_bit);
-    if (!X || !sX || !alpha || !loss || !best_alpha || !best_clip)
-        return fail(AWQ_ERR_ARG, "NULL pointer");
-    if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
-    if (N < 1 || N > (int64_t(1) << 30)) return fail(AWQ_ERR_ARG, "bad N=%lld", (long long)N);
+    if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
+                                             w_bit, quant, loss_row))
+        return s;
+    if (!alpha || !loss || !best_alpha || !best_clip) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (n_alpha < 1 || n_alpha > awq::MAX_GRID) return fail(AWQ_ERR_ARG, "n_alpha=%d", n_alpha);
     if (n_clip < 0 || n_clip > awq::MAX_GRID || (n_clip > 0 && !clip))
         return fail(AWQ_ERR_ARG, "n_clip=%d", n_clip);
@@ -301,116 +414,126 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
         if (!(alpha[k] >= 0.0 && alpha[k] <= 1.0)) return fail(AWQ_ERR_ARG, "alpha[%d] out of [0,1]", k);
     for (int k = 0; k < n_clip; ++k)
         if (!(clip[k] > 0.0 && clip[k] <= 1.0)) return fail(AWQ_ERR_ARG, "clip[%d] out of (0,1]", k);
-    if (!aligned16(X) || !aligned16(sX) || (loss_row && !aligned16(loss_row)))
-        return fail(AWQ_ERR_ALIGN, "device pointer not 16-byte aligned");
     int sms;
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
     const int G = n_alpha > n_clip ? n_alpha : n_clip;
-    const int64_t nG = in / group_size;
-    const int64_t TB = (N + awq::TILE_N - 1) / awq::TILE_N;
     const int Gtot = n_alpha + n_clip;
-    size_t bytes = 0;
-    bytes += Workspace::up(sizeof(uint16_t) * N * in);
-    bytes += Workspace::up(sizeof(float) * 2 * G * in);
-    bytes += Workspace::up(awq::scale_scratch_bytes(G, in));
-    bytes += Workspace::up(sizeof(float4) * G * out * nG);
-    bytes += Workspace::up(sizeof(float) * G * TB * out);
-    bytes += Workspace::up(sizeof(double) * Gtot);
-    bytes += Workspace::up(sizeof(double) * awq::reduce_scratch_doubles(G, out));
-    bytes += Workspace::up(sizeof(int) * 8);
+    const bool asym = quant == AWQ_ASYM, w_bf16 = w_dtype == AWQ_BF16;
     Workspace ws(st);
-    if (awq_status_t s = ws.reserve(bytes)) return s;
-    uint16_t *x16 = ws.take<uint16_t>(N * in);
-    float *sn = ws.take<float>(2 * G * in);
-    char *sc_scratch = ws.take<char>(awq::scale_scratch_bytes(G, in));
-    float4 *qparam = ws.take<float4>(G * out * nG);
-    float *part = ws.take<float>(G * TB * out);
-    double *loss_d = ws.take<double>(Gtot);
-    double *blocksum = ws.take<double>(awq::reduce_scratch_doubles(G, out));
-    // [0] best alpha, [1] best clip, [2] device error word, [3] max|X| bits, [4] X exponent
-    int *flags = ws.take<int>(8);
-    AWQ_CUDA(cudaMemsetAsync(flags, 0, sizeof(int) * 8, st));
-
-    AWQ_CUDA(awq::launch_x_to_f16(X, x_dtype == AWQ_BF16, N * in, reinterpret_cast<unsigned *>(flags + 3),
-                                  flags + 4, x16, st));
-    awq::SearchArgs a{};
-    a.w_bf16 = w_dtype == AWQ_BF16;
-    a.O = out;
-    a.I = in;
-    a.N = N;
-    a.gs = group_size;
-    a.part = part;
-    a.err = flags + 2;
-    awq::SearchMaps maps;
-
+    SearchBufs b;
+    double *loss_d;
+    if (awq_status_t s = reserve_search(ws, &b, out, in, N, group_size, G, Gtot, &loss_d)) return s;
+    AWQ_CUDA(cudaMemsetAsync(b.flags, 0, sizeof(int) * 8, st));
+    AWQ_CUDA(awq::launch_x_to_f16(X, x_dtype == AWQ_BF16, N * in,
+                                  reinterpret_cast<unsigned *>(b.flags + 3), b.flags + 4, b.x16, st));
+    kt_reset(1);
     // Phase 1: the alpha grid (clip 1).
     awq::GridParams ap{}, cp{};
     for (int k = 0; k < n_alpha; ++k) {
         ap.value[k] = alpha[k];
         cp.value[k] = 1.0;
     }
-    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_alpha, nullptr, sn, sc_scratch, st));
-    AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM, sn,
-                                      cp, n_alpha, qparam, st));
-    a.G = n_alpha;
-    a.clamp = quant == AWQ_ASYM;
-    if (awq_status_t s = make_search_maps(&maps, x16, N, W, a.w_bf16, out, in, sn, qparam, n_alpha,
-                                          group_size))
+    if (awq_status_t s = search_phase(b, W, w_bf16, out, in, N, sX, group_size, w_bit, asym, ap,
+                                      nullptr, cp, n_alpha, loss_d, loss_row, sms, st))
         return s;
-    kt_reset(1);
-    kt_begin(1, st);
-    AWQ_CUDA(awq::launch_search(a, maps, sms, st));
-    kt_end(1, st);
-    AWQ_CUDA(awq::launch_reduce_loss(part, n_alpha, TB, out, N, flags + 4, loss_d, loss_row, blocksum,
-                                     st));
-    AWQ_CUDA(awq::launch_argmin(loss_d, n_alpha, flags + 0, st));
-
+    AWQ_CUDA(awq::launch_argmin(loss_d, n_alpha, b.flags + 0, st));
     // Phase 2: the clip grid at alpha*.
     if (n_clip > 0) {
         awq::GridParams cp2{};
         for (int k = 0; k < n_clip; ++k) cp2.value[k] = clip[k];
-        AWQ_CUDA(awq::launch_scale_table(sX, in, ap, n_clip, flags + 0, sn, sc_scratch, st));
-        AWQ_CUDA(awq::launch_group_params(W, a.w_bf16, out, in, group_size, quant == AWQ_ASYM,
-                                          sn, cp2, n_clip, qparam, st));
-        a.G = n_clip;
-        a.clamp = true;
-        if (awq_status_t s = make_search_maps(&maps, x16, N, W, a.w_bf16, out, in, sn, qparam,
-                                              n_clip, group_size))
+        if (awq_status_t s = search_phase(
+                b, W, w_bf16, out, in, N, sX, group_size, w_bit, asym, ap, b.flags + 0, cp2, n_clip,
+                loss_d + n_alpha, loss_row ? loss_row + static_cast<int64_t>(n_alpha) * out : nullptr,
+                sms, st))
             return s;
-        kt_begin(1, st);
-        AWQ_CUDA(awq::launch_search(a, maps, sms, st));
-        kt_end(1, st);
-        AWQ_CUDA(awq::launch_reduce_loss(part, n_clip, TB, out, N, flags + 4, loss_d + n_alpha,
-                                         loss_row ? loss_row + static_cast<int64_t>(n_alpha) * out
-                                                  : nullptr,
-                                         blocksum, st));
-        AWQ_CUDA(awq::launch_argmin(loss_d + n_alpha, n_clip, flags + 1, st));
+        AWQ_CUDA(awq::launch_argmin(loss_d + n_alpha, n_clip, b.flags + 1, st));
     }
-
     int hflags[4];
     AWQ_CUDA(cudaMemcpyAsync(loss, loss_d, sizeof(double) * Gtot, cudaMemcpyDeviceToHost, st));
-    AWQ_CUDA(cudaMemcpyAsync(hflags, flags, sizeof(int) * 4, cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaMemcpyAsync(hflags, b.flags, sizeof(int) * 4, cudaMemcpyDeviceToHost, st));
     AWQ_CUDA(cudaStreamSynchronize(st));
-    if (hflags[2] != 0)
-        return fail(AWQ_ERR_TIMEOUT, "search kernel: a bounded wait gave up (device error %d)", hflags[2]);
+    if (awq_status_t s = device_error(hflags[2], "search kernel")) return s;
     *best_alpha = hflags[0];
     *best_clip = n_clip > 0 ? hflags[1] : -1;
     return AWQ_OK;
 }
 
-awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, const float *sX,
-                           double alpha, double clip, int group_size, int quant, uint32_t *qweight,
-                           uint16_t *scales, uint32_t *zeros, uint16_t *s16, float *scales_f32,
-                           void *stream) {
+awq_status_t awq_search_points(const void *W, int w_dtype, int64_t out, int64_t in, const void *X,
+                               int x_dtype, int64_t N, const float *sX, int group_size, int w_bit,
+                               int quant, const double *alpha, const double *clip, int n_points,
+                               double *loss, float *loss_row, int *best, void *stream) {
+    g_last_error.clear();
+    if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
+                                             w_bit, quant, loss_row))
+        return s;
+    if (!alpha || !clip || !loss || !best) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (n_points < 1 || n_points > AWQ_MAX_POINTS) return fail(AWQ_ERR_ARG, "n_points=%d", n_points);
+    for (int k = 0; k < n_points; ++k) {
+        if (!(alpha[k] >= 0.0 && alpha[k] <= 1.0)) return fail(AWQ_ERR_ARG, "alpha[%d] out of [0,1]", k);
+        if (!(clip[k] > 0.0 && clip[k] <= 1.0)) return fail(AWQ_ERR_ARG, "clip[%d] out of (0,1]", k);
+    }
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int G = n_points < awq::MAX_GRID ? n_points : awq::MAX_GRID;
+    const bool asym = quant == AWQ_ASYM, w_bf16 = w_dtype == AWQ_BF16;
+    Workspace ws(st);
+    SearchBufs b;
+    double *loss_d;
+    if (awq_status_t s = reserve_search(ws, &b, out, in, N, group_size, G, n_points, &loss_d)) return s;
+    AWQ_CUDA(cudaMemsetAsync(b.flags, 0, sizeof(int) * 8, st));
+    AWQ_CUDA(awq::launch_x_to_f16(X, x_dtype == AWQ_BF16, N * in,
+                                  reinterpret_cast<unsigned *>(b.flags + 3), b.flags + 4, b.x16, st));
+    kt_reset(1);
+    for (int k0 = 0; k0 < n_points; k0 += awq::MAX_GRID) {
+        const int g = n_points - k0 < awq::MAX_GRID ? n_points - k0 : awq::MAX_GRID;
+        awq::GridParams ap{}, cp{};
+        for (int k = 0; k < g; ++k) {
+            ap.value[k] = alpha[k0 + k];
+            cp.value[k] = clip[k0 + k];
+        }
+        if (awq_status_t s = search_phase(b, W, w_bf16, out, in, N, sX, group_size, w_bit, asym, ap,
+                                          nullptr, cp, g, loss_d + k0,
+                                          loss_row ? loss_row + static_cast<int64_t>(k0) * out : nullptr,
+                                          sms, st))
+            return s;
+    }
+    AWQ_CUDA(awq::launch_argmin(loss_d, n_points, b.flags + 0, st));
+    int hflags[4];
+    AWQ_CUDA(cudaMemcpyAsync(loss, loss_d, sizeof(double) * n_points, cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaMemcpyAsync(hflags, b.flags, sizeof(int) * 4, cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaStreamSynchronize(st));
+    if (awq_status_t s = device_error(hflags[2], "search kernel")) return s;
+    *best = hflags[0];
+    return AWQ_OK;
+}
+
+awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in, const float *sX,
+                            double alpha, double clip, const uint8_t *clip_idx,
+                            const double *clip_grid, int n_clip, int group_size, int w_bit,
+                            int quant, uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
+                            uint16_t *s16, float *scales_f32, void *stream) {
     g_last_error.clear();
     if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
+    if (w_bit != 3 && w_bit != 4) return fail(AWQ_ERR_UNSUPPORTED, "w_bit %d (3 or 4)", w_bit);
     if (!sX || !qweight || !scales || !s16) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (quant == AWQ_ASYM && !zeros) return fail(AWQ_ERR_ARG, "zeros required for AWQ_ASYM");
     if (quant == AWQ_SYM && zeros) return fail(AWQ_ERR_ARG, "zeros must be NULL for AWQ_SYM");
     if (!(alpha >= 0.0 && alpha <= 1.0)) return fail(AWQ_ERR_ARG, "alpha out of [0,1]");
-    if (!(clip > 0.0 && clip <= 1.0)) return fail(AWQ_ERR_ARG, "clip out of (0,1]");
+    awq::GridParams cg{};
+    if (clip_idx) {
+        if (!clip_grid || n_clip < 1 || n_clip > awq::MAX_GRID)
+            return fail(AWQ_ERR_ARG, "per-group clip needs a host grid of 1..%d ratios", awq::MAX_GRID);
+        for (int k = 0; k < n_clip; ++k) {
+            if (!(clip_grid[k] > 0.0 && clip_grid[k] <= 1.0))
+                return fail(AWQ_ERR_ARG, "clip_grid[%d] out of (0,1]", k);
+            cg.value[k] = clip_grid[k];
+        }
+    } else if (!(clip > 0.0 && clip <= 1.0)) {
+        return fail(AWQ_ERR_ARG, "clip out of (0,1]");
+    }
     if (!aligned16(sX) || !aligned16(qweight) || !aligned16(s16) ||
         (scales_f32 && (reinterpret_cast<uintptr_t>(scales_f32) & 3u)) ||
         (reinterpret_cast<uintptr_t>(scales) & 1u) || (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)))
@@ -431,10 +554,92 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, 
     if (zeros) AWQ_CUDA(cudaMemsetAsync(zeros, 0, sizeof(uint32_t) * out * ((nG + 7) / 8), st));
     kt_reset(2);
     kt_begin(2, st);
-    AWQ_CUDA(awq::launch_pack(W, w_dtype == AWQ_BF16, out, in, group_size, quant == AWQ_ASYM, clip,
-                              sn, qweight, scales, zeros, s16, scales_f32, st));
+    AWQ_CUDA(awq::launch_pack(W, w_dtype == AWQ_BF16, out, in, group_size, quant == AWQ_ASYM, w_bit,
+                              clip_idx ? 1.0 : clip, clip_idx, cg, sn, qweight, scales, zeros, s16,
+                              scales_f32, st));
     kt_end(2, st);
     return AWQ_OK;
+}
+
+awq_status_t awq_group_clip(const void *W, int w_dtype, int64_t out, int64_t in, const void *X,
+                            int x_dtype, int64_t N, const float *sX, double alpha, int group_size,
+                            int w_bit, int quant, const double *clip_grid, int n_clip,
+                            uint8_t *clip_idx, float *err, void *stream) {
+    g_last_error.clear();
+    if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
+                                             w_bit, quant, err))
+        return s;
+    if (N > (int64_t(1) << 26)) return fail(AWQ_ERR_UNSUPPORTED, "N above 2^26 for the group clip");
+    if (!clip_grid || !clip_idx) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!(alpha >= 0.0 && alpha <= 1.0)) return fail(AWQ_ERR_ARG, "alpha out of [0,1]");
+    if (n_clip < 1 || n_clip > awq::MAX_GRID) return fail(AWQ_ERR_ARG, "n_clip=%d", n_clip);
+    awq::GridParams cg{};
+    for (int k = 0; k < n_clip; ++k) {
+        if (!(clip_grid[k] > 0.0 && clip_grid[k] <= 1.0))
+            return fail(AWQ_ERR_ARG, "clip_grid[%d] out of (0,1]", k);
+        cg.value[k] = clip_grid[k];
+    }
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(float) * 2 * in) +
+                                    Workspace::up(awq::scale_scratch_bytes(1, in)) +
+                                    Workspace::up(sizeof(double) * awq::gclip_scratch_doubles(in, group_size))))
+        return s;
+    float *sn = ws.take<float>(2 * in);
+    char *sc_scratch = ws.take<char>(awq::scale_scratch_bytes(1, in));
+    double *H = ws.take<double>(awq::gclip_scratch_doubles(in, group_size));
+    awq::GridParams ap{};
+    ap.value[0] = alpha;
+    AWQ_CUDA(awq::launch_scale_table(sX, in, ap, 1, nullptr, sn, sc_scratch, st));
+    AWQ_CUDA(awq::launch_group_clip(W, w_dtype == AWQ_BF16, out, in, X, x_dtype == AWQ_BF16, N, sn,
+                                    group_size, quant == AWQ_ASYM, w_bit, cg, n_clip, H, clip_idx,
+                                    err, st));
+    return AWQ_OK;
+}
+
+awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, const float *sX,
+                           double alpha, double clip, int group_size, int quant, uint32_t *qweight,
+                           uint16_t *scales, uint32_t *zeros, uint16_t *s16, float *scales_f32,
+                           void *stream) {
+    return awq_pack_quant(W, w_dtype, out, in, sX, alpha, clip, nullptr, nullptr, 0, group_size, 4,
+                          quant, qweight, scales, zeros, s16, scales_f32, stream);
+}
+
+awq_status_t awq_fold_scale(const void *P, int p_dtype, int64_t rows, int64_t cols,
+                            const uint16_t *s16, void *out, void *stream) {
+    g_last_error.clear();
+    if (!P || !s16 || !out) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!valid_dtype(p_dtype)) return fail(AWQ_ERR_ARG, "bad p_dtype %d", p_dtype);
+    if (rows < 1 || cols < 1) return fail(AWQ_ERR_ARG, "bad shape rows=%lld cols=%lld", (long long)rows, (long long)cols);
+    const uintptr_t am = p_dtype == AWQ_BF16 ? 1u : 3u;
+    if ((reinterpret_cast<uintptr_t>(P) & am) || (reinterpret_cast<uintptr_t>(out) & am) ||
+        (reinterpret_cast<uintptr_t>(s16) & 1u))
+        return fail(AWQ_ERR_ALIGN, "misaligned pointer");
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    AWQ_CUDA(awq::launch_fold_scale(P, p_dtype == AWQ_BF16, rows, cols, s16, out,
+                                    static_cast<cudaStream_t>(stream)));
+    return AWQ_OK;
+}
+
+awq_status_t awq_wait_selftest(int64_t limit_cycles, int arrive, void *stream) {
+    g_last_error.clear();
+    if (limit_cycles < 1 || limit_cycles > awq::AWQ_DEFAULT_WAIT_CYCLES)
+        return fail(AWQ_ERR_ARG, "limit_cycles out of [1, %lld]", (long long)awq::AWQ_DEFAULT_WAIT_CYCLES);
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    Workspace ws(st);
+    if (awq_status_t s = ws.reserve(Workspace::up(sizeof(int)))) return s;
+    int *err = ws.take<int>(1);
+    AWQ_CUDA(cudaMemsetAsync(err, 0, sizeof(int), st));
+    AWQ_CUDA(awq::launch_wait_selftest(limit_cycles, arrive != 0, err, st));
+    int h = 0;
+    AWQ_CUDA(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, st));
+    AWQ_CUDA(cudaStreamSynchronize(st));
+    return device_error(h, "wait self-test");
 }
 
 awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
@@ -442,7 +647,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
                               const uint32_t *zeros, const uint16_t *s16, int group_size,
                               uint16_t *y, void *stream) {
     g_last_error.clear();
-    if (!x || !qweight || !scales || !s16 || !y) return fail(AWQ_ERR_ARG, "NULL pointer");
+    if (!x || !qweight || !scales || !y) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (M < 1 || in < 1 || out < 1) return fail(AWQ_ERR_ARG, "bad shape");
     if (group_size != 32 && group_size != 64 && group_size != 128)
         return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
@@ -451,7 +656,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
         return fail(AWQ_ERR_UNSUPPORTED, "in=%lld is not a multiple of group_size %d", (long long)in, group_size);
     if (in > 49152) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld above 49152", (long long)in);
     if (!aligned16(x) || !aligned16(qweight) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
-        (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)) || !aligned16(s16) ||
+        (zeros && (reinterpret_cast<uintptr_t>(zeros) & 3u)) || (s16 && !aligned16(s16)) ||
         (reinterpret_cast<uintptr_t>(y) & 1u))
         return fail(AWQ_ERR_ALIGN, "misaligned pointer");
     int sms;

@@ -12,7 +12,18 @@ namespace awq {
 void set_last_error(const char *msg);
 
 constexpr int STATS_CHUNK = 128;   // tokens per fp64 partial sum of mean|X|
+constexpr int64_t STATS_MAX_GRID_Y = 65535;   // chunks beyond this are strided over the grid
+
+// Optional CUDA-event timing of an entry point's main kernels (awq_set_kernel_timing):
+// kt_reset clears the record of `kind`, kt_begin / kt_end bracket launches on `st`.
+void kt_reset(int kind);
+void kt_begin(int kind, cudaStream_t st);
+void kt_end(int kind, cudaStream_t st);
 constexpr int MAX_GRID = 64;       // grid points per search phase
+
+// Default bound of an in-kernel mbarrier wait: ~2 s of SM clock at 2 GHz, far
+// above any legitimate wait in these kernels.
+constexpr long long AWQ_DEFAULT_WAIT_CYCLES = 4000000000LL;
 
 // Search tile shape: 128 output rows x 512 tokens per work unit, K slabs of 64.
 constexpr int TILE_O = 128;
@@ -42,10 +53,13 @@ cudaError_t launch_scale_table(const float *sX, int64_t I, const GridParams &alp
                                const int *best_idx, float *sn, void *scratch, cudaStream_t st);
 
 // ---- per-(grid point, group, row) quantiser parameters {Delta, 1/Delta, -qhi, -qlo},
-// layout qparam[g][group][row] (rows fastest)
+// layout qparam[g][group][row] (rows fastest).  Also picks each grid point's
+// power-of-two range scale 2^k of dW (dw_exp[g] = k, device), multiplying the
+// -1/s rows of sn by it; dw_bits: G words of device scratch.
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
-                                bool asym, const float *sn, const GridParams &clip, int G,
-                                float4 *qparam, cudaStream_t st);
+                                bool asym, int wbit, float *sn, const GridParams &clip,
+                                int G, float4 *qparam, unsigned *dw_bits, int *dw_exp,
+                                cudaStream_t st);
 
 // ---- fused search
 // Tensor maps of the kernel's four inputs:
@@ -64,6 +78,7 @@ struct SearchArgs {
     bool clamp;                 // asymmetric or clipped: clamp codes to [qlo, qhi]
     float *part;                // [G][TB][O]
     int *err;
+    long long wait;             // bound of every mbarrier wait, in SM clock cycles
 };
 cudaError_t launch_search(const SearchArgs &a, const SearchMaps &maps, int num_sms,
                           cudaStream_t st);
@@ -71,16 +86,20 @@ cudaError_t launch_search(const SearchArgs &a, const SearchMaps &maps, int num_s
 // ---- loss reduction and selection
 // blocksum: scratch of reduce_scratch_doubles(G, O) doubles.
 int64_t reduce_scratch_doubles(int G, int64_t O);
-// Row sums are multiplied by 2^(2 * *x_exp) (the exact undo of X's fp16 scaling).
+// Row sums of grid point g are multiplied by 2^(-2 * (*x_exp + dw_exp[g])) (the exact
+// undo of the power-of-two scales of X and dW in the contraction).
 cudaError_t launch_reduce_loss(const float *part, int G, int64_t TB, int64_t O, int64_t N,
-                               const int *x_exp, double *loss, float *loss_row, double *blocksum,
-                               cudaStream_t st);
+                               const int *x_exp, const int *dw_exp, double *loss, float *loss_row,
+                               double *blocksum, cudaStream_t st);
 cudaError_t launch_argmin(const double *loss, int G, int *best, cudaStream_t st);
 
 // ---- packing
+// clip_idx (optional, [O][I/gs] device): each group's index into clip_grid, used
+// instead of the layer ratio `clip`.
 cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs, bool asym,
-                        double clip, const float *s, uint32_t *qweight, uint16_t *scales,
-                        uint32_t *zeros, uint16_t *s16, float *scales_f32, cudaStream_t st);
+                        int wbit, double clip, const uint8_t *clip_idx, const GridParams &clip_grid,
+                        const float *s, uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
+                        uint16_t *s16, float *scales_f32, cudaStream_t st);
 
 // ---- W4A16 apply on the tensor cores (M >= 5)
 struct TcMaps {
@@ -110,5 +129,24 @@ cudaError_t launch_w4a16_stream(const uint16_t *x, int64_t M, int64_t I, int64_t
 cudaError_t launch_w4a16(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                          const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
                          const uint16_t *s16, int gs, uint16_t *y, cudaStream_t st);
+
+// ---- per-group clip choice: Gram matrices of X per group (H: gclip_scratch_doubles
+// device doubles), then for every (row, group) the first ratio of `grid` that
+// minimises the group's output error; best [O][I/gs] u8, err (optional) [O][I/gs][n_clip].
+int64_t gclip_scratch_doubles(int64_t I, int gs);
+cudaError_t launch_group_clip(const void *W, bool w_bf16, int64_t O, int64_t I, const void *X,
+                              bool x_bf16, int64_t N, const float *s, int gs, bool asym, int wbit,
+                              const GridParams &grid, int n_clip, double *H, uint8_t *best,
+                              float *err, cudaStream_t st);
+
+// ---- bounded-wait self-test: one CTA waits on an mbarrier (arrived on only if
+// `arrive`) with a limit of `limit` cycles; a wait that gives up writes the
+// timeout code to *err.
+cudaError_t launch_wait_selftest(long long limit, bool arrive, int *err, cudaStream_t st);
+
+// ---- fold of 1/s into the previous operator: out[r][c] = P[r][c] / s16[r]
+// (one IEEE fp32 division, then bf16 rounding when bf16).
+cudaError_t launch_fold_scale(const void *P, bool bf16, int64_t R, int64_t C, const uint16_t *s16,
+                              void *out, cudaStream_t st);
 
 }  // namespace awq

@@ -77,8 +77,12 @@ extern "C" awq_status_t awq_act_stats_noalloc(const void *X, int x_dtype, int64_
     if (e != cudaSuccess) return reject(AWQ_ERR_CUDA, cudaGetErrorString(e));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // The partial kernel overwrites every partial it uses, so nothing needs clearing.
+    // Timing (when enabled) is recorded as kind 0, like awq_act_stats.
+    awq::kt_reset(0);
+    awq::kt_begin(0, st);
     e = awq::launch_stats_partial(X, x_dtype == AWQ_BF16, N, in, part, st);
     if (e == cudaSuccess) e = awq::launch_stats_final(part, N, in, clamp_min, sX, st);
     if (e != cudaSuccess) return reject(AWQ_ERR_CUDA, cudaGetErrorString(e));
+    awq::kt_end(0, st);
     return AWQ_OK;
 }

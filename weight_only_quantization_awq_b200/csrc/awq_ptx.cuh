@@ -9,10 +9,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "awq_internal.h"
+
 namespace awq {
 
 // ~2 s at 2 GHz: far above any legitimate wait in these kernels.
-constexpr long long AWQ_WAIT_CYCLES = 4000000000LL;
+constexpr long long AWQ_WAIT_CYCLES = AWQ_DEFAULT_WAIT_CYCLES;
 
 // Error codes written to the device error word.
 constexpr int DEV_ERR_TIMEOUT = 5;
@@ -54,15 +56,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// CTA abort flag is (or becomes) set, or after AWQ_WAIT_CYCLES, in which case
-// it sets the abort flag itself.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// CTA abort flag is (or becomes) set, or after `limit` SM clock cycles (a
+// kernel argument, AWQ_WAIT_CYCLES by default), in which case it sets the abort
+// flag itself.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                          long long limit = AWQ_WAIT_CYCLES) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > AWQ_WAIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             return false;
         }
@@ -72,14 +76,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // As mbar_wait, but sleeping between polls: for waits that usually last a
 // whole work unit, so the waiting warps do not take issue slots from the rest.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity,
-                                                volatile int *abort_flag) {
+                                                volatile int *abort_flag,
+                                                long long limit = AWQ_WAIT_CYCLES) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         __nanosleep(256);
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > AWQ_WAIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             return false;
         }
@@ -87,10 +92,11 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity,
 }
 
 // Same, ignoring the abort flag (used only to drain in-flight copies on exit).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
+                                                long long limit = AWQ_WAIT_CYCLES) {
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > AWQ_WAIT_CYCLES) return false;
+        if (clock64() - t0 > limit) return false;
     }
     return true;
 }

@@ -6,6 +6,7 @@
 //           (max - min) / 15 with zero point z = clamp(rint(-min/Delta), 0, 15)
 //           for the asymmetric one (AWQ guide, section 三, step 4; paper
 //           summary, Method, first equation); clip ratios scale the bounds.
+//           At w_bit = 3 the constants are 3 (codes [-4, 3]) and 7 ([0, 7]).
 //
 // Everything that decides an integer (Delta, z, codes) uses IEEE fp32
 // operations with explicit rounding intrinsics, so no FMA contraction or
@@ -90,10 +91,14 @@ __device__ __forceinline__ float safe_rcp(float d) {
 // registers and loops over the G grid points; each grid point's s values for
 // the group are broadcast from shared memory.  Output layout qparam[g][j][o]
 // (rows fastest) so the writes coalesce.
+// It also bounds |dW| = |(q - z)*Delta/s - W| over the layer per grid point:
+//     |dW[o, i]| <= max_group |W| + 2^w_bit * Delta / min_group s,
+// folded into dw_bits[g] with an atomic max on the bit pattern (>= 0).
 template <bool WBF16, int GS>
 __global__ void __launch_bounds__(128) group_params_kernel(
-    const void *__restrict__ W, int64_t O, int64_t I, bool asym, const float *__restrict__ sn,
-    GridParams clip, int G, float4 *__restrict__ qparam) {
+    const void *__restrict__ W, int64_t O, int64_t I, bool asym, int wbit,
+    const float *__restrict__ sn, GridParams clip, int G, float4 *__restrict__ qparam,
+    unsigned *__restrict__ dw_bits) {
     __shared__ __align__(16) float s_sm[MAX_GRID][GS];
     const int64_t j = blockIdx.y;
     const int64_t nG = I / GS;
@@ -102,6 +107,7 @@ __global__ void __launch_bounds__(128) group_params_kernel(
     __syncthreads();
     const int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (o >= O) return;
+    const unsigned live = __activemask();
     constexpr int NW = WBF16 ? GS / 2 : GS;      // 32-bit words of the group
     uint32_t wr[NW];
     const uint4 *src = WBF16 ? reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(W) + o * I + j * GS)
@@ -111,15 +117,24 @@ __global__ void __launch_bounds__(128) group_params_kernel(
         const uint4 v = __ldg(src + k);
         wr[4 * k] = v.x; wr[4 * k + 1] = v.y; wr[4 * k + 2] = v.z; wr[4 * k + 3] = v.w;
     }
+    float wabs = 0.0f;                           // max |W| of the group
+#pragma unroll
+    for (int e = 0; e < GS; ++e) {
+        if constexpr (WBF16)
+            wabs = fmaxf(wabs, fabsf(__uint_as_float((e & 1) ? (wr[e >> 1] & 0xFFFF0000u) : (wr[e >> 1] << 16))));
+        else
+            wabs = fmaxf(wabs, fabsf(__uint_as_float(wr[e])));
+    }
     for (int g = 0; g < G; ++g) {
         // four independent max / min chains (max and min are exact, so the split
         // changes no result), merged at the end
-        float mx4[4], mn4[4], am4[4];
+        float mx4[4], mn4[4], am4[4], smin4[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             mx4[k] = -3.4028234663852886e38f;
             mn4[k] = 3.4028234663852886e38f;
             am4[k] = 0.0f;
+            smin4[k] = 3.4028234663852886e38f;
         }
 #pragma unroll
         for (int e4 = 0; e4 < GS / 4; ++e4) {
@@ -134,6 +149,7 @@ __global__ void __launch_bounds__(128) group_params_kernel(
                 else
                     w = __uint_as_float(wr[e]);
                 const float wp = __fmul_rn(w, sv[k]);
+                smin4[k] = fminf(smin4[k], sv[k]);
                 if (asym) {
                     mx4[k] = fmaxf(mx4[k], wp);
                     mn4[k] = fminf(mn4[k], wp);
@@ -148,29 +164,63 @@ __global__ void __launch_bounds__(128) group_params_kernel(
         const double r = clip.value[g];
         float D, qlo, qhi;
         if (!asym) {
-            D = __fdiv_rn(clip_bound(amax, r), 7.0f);
-            qlo = -8.0f;
-            qhi = 7.0f;
+            const float top = static_cast<float>((1 << (wbit - 1)) - 1);   // 7 or 3
+            D = __fdiv_rn(clip_bound(amax, r), top);
+            qlo = -top - 1.0f;
+            qhi = top;
         } else {
+            const float top = static_cast<float>((1 << wbit) - 1);         // 15 or 7
             const float hi = clip_bound(mx, r), lo = clip_bound(mn, r);
-            D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+            D = __fdiv_rn(__fsub_rn(hi, lo), top);
             float z = 0.0f;
-            if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+            if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), top);
             qlo = -z;
-            qhi = 15.0f - z;
+            qhi = top - z;
             if (D == 0.0f) qhi = 0.0f;
         }
         // {Delta, 1/Delta, -qhi, -qlo}: the search kernel works with -q.
         qparam[(static_cast<int64_t>(g) * nG + j) * O + o] = make_float4(D, safe_rcp(D), -qhi, -qlo);
+        const float smin = fminf(fminf(smin4[0], smin4[1]), fminf(smin4[2], smin4[3]));
+        const float bound = wabs + static_cast<float>(1 << wbit) * D / smin;
+        const unsigned b = (bound >= 0.0f && bound < 3.0e38f) ? __float_as_uint(bound) : 0x7F000000u;
+        const unsigned wmax = __reduce_max_sync(live, b);
+        if ((threadIdx.x & 31) == __ffs(live) - 1) atomicMax(&dw_bits[g], wmax);
     }
 }
 
+// dW goes to fp16 for the tensor cores.  Grid point g's bound B on |dW| picks
+// k with B * 2^k in [2^14, 2^15) (|k| <= 60); the -1/s row of the scale table
+// is multiplied by 2^k (exact), so the search kernel forms 2^k * dW at no cost,
+// and the loss reduction multiplies by 2^-2k.  Without it, a layer of small
+// weights would put dW into fp16's subnormal range.
+__global__ void __launch_bounds__(256) dw_scale_kernel(int64_t I, const unsigned *__restrict__ dw_bits,
+                                                       float *__restrict__ sn, int *__restrict__ dw_exp) {
+    const int g = blockIdx.y;
+    const float b = __uint_as_float(dw_bits[g]);
+    int k = 0;
+    if (b > 0.0f) {
+        int e;
+        frexpf(b, &e);                            // b = f * 2^e, f in [0.5, 1)
+        k = 15 - e;
+        k = k < -60 ? -60 : (k > 60 ? 60 : k);
+    }
+    const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < I) {
+        float *row = sn + (2 * static_cast<int64_t>(g) + 1) * I;
+        row[i] = ldexpf(row[i], k);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) dw_exp[g] = k;
+}
+
 cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I, int gs,
-                                bool asym, const float *sn, const GridParams &clip, int G,
-                                float4 *qparam, cudaStream_t st) {
+                                bool asym, int wbit, float *sn, const GridParams &clip,
+                                int G, float4 *qparam, unsigned *dw_bits, int *dw_exp,
+                                cudaStream_t st) {
+    cudaError_t e0 = cudaMemsetAsync(dw_bits, 0, sizeof(unsigned) * G, st);
+    if (e0 != cudaSuccess) return e0;
     const dim3 grid(static_cast<unsigned>((O + 127) / 128), static_cast<unsigned>(I / gs));
 #define AWQ_GP(WB, GSZ) \
-    group_params_kernel<WB, GSZ><<<grid, 128, 0, st>>>(W, O, I, asym, sn, clip, G, qparam)
+    group_params_kernel<WB, GSZ><<<grid, 128, 0, st>>>(W, O, I, asym, wbit, sn, clip, G, qparam, dw_bits)
     if (w_bf16) {
         if (gs == 32) AWQ_GP(true, 32);
         else if (gs == 64) AWQ_GP(true, 64);
@@ -181,6 +231,10 @@ cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I
         else AWQ_GP(false, 128);
     }
 #undef AWQ_GP
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dw_scale_kernel<<<dim3(static_cast<unsigned>((I + 255) / 256), static_cast<unsigned>(G)), 256, 0, st>>>(
+        I, dw_bits, sn, dw_exp);
     return cudaGetLastError();
 }
 
@@ -195,7 +249,9 @@ constexpr int PACK_THREADS = 128;
 
 template <bool WBF16>
 __global__ void __launch_bounds__(PACK_THREADS) pack_kernel(const void *__restrict__ W, int O, int I,
-                                                            int gs, bool asym, double clip,
+                                                            int gs, bool asym, int wbit, double clip,
+                                                            const uint8_t *__restrict__ clip_idx,
+                                                            GridParams clip_grid,
                                                             const float *__restrict__ s,
                                                             uint32_t *__restrict__ qweight,
                                                             uint16_t *__restrict__ scales,
@@ -283,15 +339,20 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_kernel(const void *__restri
         gmn = fminf(gmn, __shfl_xor_sync(0xffffffffu, gmn, off));
         gam = fmaxf(gam, __shfl_xor_sync(0xffffffffu, gam, off));
     }
+    // the group's clip ratio: one per layer, or its own entry of the per-group choice
+    const int jg = active ? w0 / wpg : 0;
+    if (clip_idx && active) clip = clip_grid.value[clip_idx[static_cast<int64_t>(o) * nG + jg]];
+    const float stop = static_cast<float>((1 << (wbit - 1)) - 1);   // symmetric top code: 7 or 3
+    const float atop = static_cast<float>((1 << wbit) - 1);         // asymmetric top code: 15 or 7
     float D, z = 0.0f;
     if (!asym) {
         const float a = clip == 1.0 ? gam : __double2float_rn(__dmul_rn((double)gam, clip));
-        D = __fdiv_rn(a, 7.0f);
+        D = __fdiv_rn(a, stop);
     } else {
         const float hi = clip == 1.0 ? gmx : __double2float_rn(__dmul_rn((double)gmx, clip));
         const float lo = clip == 1.0 ? gmn : __double2float_rn(__dmul_rn((double)gmn, clip));
-        D = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
-        if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), 15.0f);
+        D = __fdiv_rn(__fsub_rn(hi, lo), atop);
+        if (D != 0.0f) z = fminf(fmaxf(rintf(__fdiv_rn(-lo, D)), 0.0f), atop);
     }
     // q = rint(RN(W'/Delta)) from the reciprocal product W' * RN(1/Delta): every
     // decision that survives the clamp has |W'/Delta| <= 15.5, where the product
@@ -315,7 +376,8 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_kernel(const void *__restri
         uint32_t wd = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float c = asym ? fminf(fmaxf(q[e] + z, 0.0f), 15.0f) : fminf(fmaxf(q[e], -8.0f), 7.0f) + 8.0f;
+            const float c = asym ? fminf(fmaxf(q[e] + z, 0.0f), atop)
+                                 : fminf(fmaxf(q[e], -stop - 1.0f), stop) + 8.0f;
             wd |= (static_cast<uint32_t>(static_cast<int>(c)) & 0xFu) << (4 * e);
         }
         word[k] = wd;
@@ -340,17 +402,20 @@ __global__ void __launch_bounds__(PACK_THREADS) pack_kernel(const void *__restri
 }
 
 cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs, bool asym,
-                        double clip, const float *s, uint32_t *qweight, uint16_t *scales,
-                        uint32_t *zeros, uint16_t *s16, float *scales_f32, cudaStream_t st) {
+                        int wbit, double clip, const uint8_t *clip_idx, const GridParams &clip_grid,
+                        const float *s, uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
+                        uint16_t *s16, float *scales_f32, cudaStream_t st) {
     const int64_t wpr = I / 8;
     const dim3 grid(static_cast<unsigned>(O),
                     static_cast<unsigned>((wpr / PACK_PW + PACK_THREADS - 1) / PACK_THREADS));
     if (w_bf16)
         pack_kernel<true><<<grid, PACK_THREADS, 0, st>>>(W, static_cast<int>(O), static_cast<int>(I), gs, asym,
-                                                         clip, s, qweight, scales, zeros, s16, scales_f32);
+                                                         wbit, clip, clip_idx, clip_grid, s, qweight,
+                                                         scales, zeros, s16, scales_f32);
     else
         pack_kernel<false><<<grid, PACK_THREADS, 0, st>>>(W, static_cast<int>(O), static_cast<int>(I), gs, asym,
-                                                          clip, s, qweight, scales, zeros, s16, scales_f32);
+                                                          wbit, clip, clip_idx, clip_grid, s, qweight,
+                                                          scales, zeros, s16, scales_f32);
     return cudaGetLastError();
 }
 

@@ -14,6 +14,7 @@ constexpr int RED_THREADS = 256;
 __global__ void __launch_bounds__(RED_THREADS) reduce_rows_kernel(const float *__restrict__ part,
                                                                   int64_t TB, int64_t O,
                                                                   const int *__restrict__ x_exp,
+                                                                  const int *__restrict__ dw_exp,
                                                                   float *__restrict__ loss_row,
                                                                   double *__restrict__ blocksum) {
     __shared__ double red[RED_THREADS];
@@ -23,7 +24,7 @@ __global__ void __launch_bounds__(RED_THREADS) reduce_rows_kernel(const float *_
     if (o < O) {
         const float *p = part + static_cast<int64_t>(g) * TB * O + o;
         for (int64_t tb = 0; tb < TB; ++tb) v = __dadd_rn(v, static_cast<double>(p[tb * O]));
-        v = ldexp(v, 2 * *x_exp);
+        v = ldexp(v, 2 * (*x_exp - dw_exp[g]));
         if (loss_row) loss_row[static_cast<int64_t>(g) * O + o] = __double2float_rn(v);
     }
     red[threadIdx.x] = v;
@@ -65,10 +66,11 @@ int64_t reduce_scratch_doubles(int G, int64_t O) {
 }
 
 cudaError_t launch_reduce_loss(const float *part, int G, int64_t TB, int64_t O, int64_t N,
-                               const int *x_exp, double *loss, float *loss_row, double *blocksum,
-                               cudaStream_t st) {
+                               const int *x_exp, const int *dw_exp, double *loss, float *loss_row,
+                               double *blocksum, cudaStream_t st) {
     const int nblk = static_cast<int>((O + RED_THREADS - 1) / RED_THREADS);
-    reduce_rows_kernel<<<dim3(nblk, G), RED_THREADS, 0, st>>>(part, TB, O, x_exp, loss_row, blocksum);
+    reduce_rows_kernel<<<dim3(nblk, G), RED_THREADS, 0, st>>>(part, TB, O, x_exp, dw_exp, loss_row,
+                                                              blocksum);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     reduce_blocks_kernel<<<G, RED_THREADS, 0, st>>>(blocksum, nblk,

@@ -178,7 +178,7 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
     for (int64_t u = pair_id(); u < U; u += pair_count()) {
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
             const uint32_t is = it % P::IS, as = it % P::AS;
-            if (!mbar_wait(&in_full[is], (it / P::IS) & 1u, abort_flag)) return;
+            if (!mbar_wait(&in_full[is], (it / P::IS) & 1u, abort_flag, a.wait)) return;
             const uint8_t *in = in_ring + is * P::IN_STAGE;
             uint8_t *dst = a_ring + as * A_STAGE_BYTES;
             // Read all of this thread's inputs of the slab (16 weights, their s and
@@ -219,7 +219,7 @@ __device__ __forceinline__ void producer_role(const SearchArgs &a, int64_t U,
             // before lane 0's arrive.
             __syncwarp();
             if (lane == 0) mbar_arrive(&in_empty[is]);
-            if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag)) return;
+            if (!mbar_wait(&a_empty[as], ((it / P::AS) & 1u) ^ 1u, abort_flag, a.wait)) return;
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
                 const int ch = qc * 2 + (cc ^ (qc >> 1));
@@ -255,7 +255,7 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
         const int64_t nG = a.I / a.gs;
         for (int64_t kb = 0; kb < nK; ++kb, ++it) {
             const uint32_t st = it % P::IS;
-            if (!mbar_wait(&in_empty[st], ((it / P::IS) & 1u) ^ 1u, abort_flag)) {
+            if (!mbar_wait(&in_empty[st], ((it / P::IS) & 1u) ^ 1u, abort_flag, a.wait)) {
                 ok = false;
                 break;
             }
@@ -279,7 +279,7 @@ __device__ __forceinline__ void input_loader(const SearchArgs &a, const SearchMa
     // Never leave the CTA with a copy still landing in its shared memory.
 #pragma unroll
     for (int s = 0; s < P::IS; ++s)
-        if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / P::IS) & 1));
+        if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / P::IS) & 1), a.wait);
 }
 
 // Lane 0 of the TMA warp: this CTA's half (128 tokens) of each X tile for the
@@ -301,7 +301,7 @@ __device__ __forceinline__ void x_loader(const SearchArgs &a, const CUtensorMap 
         for (int64_t kb = 0; kb < nK && ok; ++kb) {
             for (int h = 0; h < un.nsub; ++h, ++it) {
                 const uint32_t stage = it % XS, phase = (it / XS) & 1u;
-                if (!mbar_wait(&x_empty[stage], phase ^ 1u, abort_flag)) {
+                if (!mbar_wait(&x_empty[stage], phase ^ 1u, abort_flag, a.wait)) {
                     ok = false;
                     break;
                 }
@@ -330,7 +330,7 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
         const Unit un = decode(u, a, OT);
         for (int64_t kb = 0; kb < nK && ok; ++kb, ++ait) {
             const uint32_t as = ait % AS;
-            if (!mbar_wait(&a_full[as], (ait / AS) & 1u, abort_flag)) {
+            if (!mbar_wait(&a_full[as], (ait / AS) & 1u, abort_flag, a.wait)) {
                 ok = false;
                 break;
             }
@@ -340,14 +340,14 @@ __device__ __forceinline__ void mma_role(const SearchArgs &a, int64_t OT, int64_
                 // each 256-column half of the accumulator is waited for separately, so
                 // this unit starts on half 0 while the epilogue still drains half 1
                 if (kb == 0) {
-                    if (!mbar_wait(&acc_empty[h], (hit[h] & 1u) ^ 1u, abort_flag)) {
+                    if (!mbar_wait(&acc_empty[h], (hit[h] & 1u) ^ 1u, abort_flag, a.wait)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                 }
                 const uint32_t xs = xit % XS;
-                if (!mbar_wait(&x_full[xs], (xit / XS) & 1u, abort_flag)) {
+                if (!mbar_wait(&x_full[xs], (xit / XS) & 1u, abort_flag, a.wait)) {
                     ok = false;
                     break;
                 }
@@ -384,7 +384,7 @@ __device__ __forceinline__ void epilogue_role(const SearchArgs &a, int64_t OT, i
         const Unit un = decode(u, a, OT);
         float sum = 0.0f;
         for (int h = 0; h < un.nsub; ++h) {
-            const bool ok = mbar_wait_sleep(&acc_full[h], hit[h] & 1u, abort_flag);
+            const bool ok = mbar_wait_sleep(&acc_full[h], hit[h] & 1u, abort_flag, a.wait);
             if (!__all_sync(0xffffffffu, ok)) return;
             tc_fence_after();
 #pragma unroll 1
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Every pair MMA has finished (the leader's last commit reaches both CTAs)
     // before TMEM is freed, and neither CTA leaves while the other may still
     // signal its barriers or read its shared memory.
-    if (warp == WARP_MMA && lane == 0) mbar_wait_drain(drain, 0);
+    if (warp == WARP_MMA && lane == 0) mbar_wait_drain(drain, 0, a.wait);
     __syncwarp();
     cluster_sync_all();
     if (threadIdx.x == 0 && *abort_flag) atomicExch(a.err, DEV_ERR_TIMEOUT);

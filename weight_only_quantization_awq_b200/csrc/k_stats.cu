@@ -21,36 +21,41 @@ __device__ __forceinline__ double abs_bf16_hi(uint32_t v) {
     return fabs(static_cast<double>(__uint_as_float(v & 0xFFFF0000u)));
 }
 
+// Chunks are dealt over gridDim.y with a stride, so any number of tokens fits
+// the grid's y limit; every chunk's partial is summed the same way whichever
+// block computes it.
 template <bool BF16>
 __global__ void __launch_bounds__(128) stats_partial_kernel(const void *__restrict__ X, int64_t N,
                                                             int64_t I, double *__restrict__ part) {
     const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // column pair
     if (q * 2 >= I) return;
-    const int64_t c = blockIdx.y;
-    const int64_t n0 = c * STATS_CHUNK;
-    const int64_t n1 = (n0 + STATS_CHUNK < N) ? n0 + STATS_CHUNK : N;
-    double a0 = 0.0, a1 = 0.0;
+    const int64_t n_chunks = (N + STATS_CHUNK - 1) / STATS_CHUNK;
     const int64_t stride = I / 2;   // column pairs per row
-    if constexpr (BF16) {
-        const uint32_t *p = reinterpret_cast<const uint32_t *>(X) + n0 * stride + q;
+    for (int64_t c = blockIdx.y; c < n_chunks; c += gridDim.y) {
+        const int64_t n0 = c * STATS_CHUNK;
+        const int64_t n1 = (n0 + STATS_CHUNK < N) ? n0 + STATS_CHUNK : N;
+        double a0 = 0.0, a1 = 0.0;
+        if constexpr (BF16) {
+            const uint32_t *p = reinterpret_cast<const uint32_t *>(X) + n0 * stride + q;
 #pragma unroll 32
-        for (int64_t n = n0; n < n1; ++n) {
-            const uint32_t v = __ldg(p);
-            p += stride;
-            a0 += abs_bf16_lo(v);
-            a1 += abs_bf16_hi(v);
-        }
-    } else {
-        const float2 *p = reinterpret_cast<const float2 *>(X) + n0 * stride + q;
+            for (int64_t n = n0; n < n1; ++n) {
+                const uint32_t v = __ldg(p);
+                p += stride;
+                a0 += abs_bf16_lo(v);
+                a1 += abs_bf16_hi(v);
+            }
+        } else {
+            const float2 *p = reinterpret_cast<const float2 *>(X) + n0 * stride + q;
 #pragma unroll 32
-        for (int64_t n = n0; n < n1; ++n) {
-            const float2 v = __ldg(p);
-            p += stride;
-            a0 += fabs(static_cast<double>(v.x));
-            a1 += fabs(static_cast<double>(v.y));
+            for (int64_t n = n0; n < n1; ++n) {
+                const float2 v = __ldg(p);
+                p += stride;
+                a0 += fabs(static_cast<double>(v.x));
+                a1 += fabs(static_cast<double>(v.y));
+            }
         }
+        reinterpret_cast<double2 *>(part + c * I)[q] = make_double2(a0, a1);
     }
-    reinterpret_cast<double2 *>(part + c * I)[q] = make_double2(a0, a1);
 }
 
 __global__ void __launch_bounds__(256) stats_final_kernel(const double *__restrict__ part,
@@ -142,7 +147,8 @@ cudaError_t launch_stats_partial(const void *X, bool x_bf16, int64_t N, int64_t 
                                  cudaStream_t st) {
     const int64_t n_chunks = (N + STATS_CHUNK - 1) / STATS_CHUNK;
     const int64_t pairs = I / 2;
-    dim3 grid(static_cast<unsigned>((pairs + 127) / 128), static_cast<unsigned>(n_chunks));
+    const int64_t gy = n_chunks < STATS_MAX_GRID_Y ? n_chunks : STATS_MAX_GRID_Y;
+    dim3 grid(static_cast<unsigned>((pairs + 127) / 128), static_cast<unsigned>(gy));
     if (x_bf16)
         stats_partial_kernel<true><<<grid, 128, 0, st>>>(X, N, I, part);
     else

@@ -61,8 +61,8 @@ __global__ void __launch_bounds__(W4_THREADS) w4a16_decode_kernel(
         float v = 0.0f;
         if (m < mt && c < I) {
             const float inv16 = j == 0 ? 1.0f : (j == 1 ? 0.0625f : (j == 2 ? 0.00390625f : 0.000244140625f));
-            v = __uint_as_float(static_cast<uint32_t>(x[(m0 + m) * I + c]) << 16) *
-                (__frcp_rn(__half2float(__ushort_as_half(s16[c]))) * inv16);
+            const float rs = s16 ? __frcp_rn(__half2float(__ushort_as_half(s16[c]))) : 1.0f;
+            v = __uint_as_float(static_cast<uint32_t>(x[(m0 + m) * I + c]) << 16) * (rs * inv16);
         }
         xsf[m * xs_floats + 2 * xs_pair_index(b, wd, j, l) + half] = v;
     }

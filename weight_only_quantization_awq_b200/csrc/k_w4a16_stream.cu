@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(GvShape<MT>::NW * 32, 1) w4a16_gemv_kernel(con
         l2_prefetch_range(a.qweight + row0 * (I / 8), static_cast<uint64_t>(nrows) * (I / 2));
         l2_prefetch_range(a.scales + row0 * nG, static_cast<uint64_t>(nrows) * nG * 2);
         if (ZEROS) l2_prefetch_range(a.zeros + row0 * nzw, static_cast<uint64_t>(nrows) * nzw * 4);
-        l2_prefetch_range(a.s16, static_cast<uint64_t>(I) * 2);
+        if (a.s16) l2_prefetch_range(a.s16, static_cast<uint64_t>(I) * 2);
         l2_prefetch_range(a.x, static_cast<uint64_t>(a.M) * I * 2);
     }
     griddep_launch_dependents();
@@ -145,7 +145,9 @@ __global__ void __launch_bounds__(GvShape<MT>::NW * 32, 1) w4a16_gemv_kernel(con
         xv = sv = make_uint4(0u, 0u, 0u, 0u);
         if (task < ntask && m < a.M && t < nch) {
             xv = __ldg(reinterpret_cast<const uint4 *>(a.x + static_cast<int64_t>(m) * I + t * 32 + wd * 8));
-            sv = __ldg(reinterpret_cast<const uint4 *>(a.s16 + t * 32 + wd * 8));
+            // no s16: x arrives already divided by s (fp16 ones leave it unchanged)
+            sv = a.s16 ? __ldg(reinterpret_cast<const uint4 *>(a.s16 + t * 32 + wd * 8))
+                       : make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
         }
     };
     uint4 xv0, sv0;

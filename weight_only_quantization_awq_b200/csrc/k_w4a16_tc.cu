@@ -58,8 +58,8 @@ __global__ void __launch_bounds__(256) xs_absmax_kernel(const uint16_t *__restri
     const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < M * I; k += step) {
         const int64_t c = k % I;
-        m = fmaxf(m, fabsf(__fdividef(__uint_as_float(static_cast<uint32_t>(x[k]) << 16),
-                                      __half2float(__ushort_as_half(s16[c])))));
+        const float xv = __uint_as_float(static_cast<uint32_t>(x[k]) << 16);
+        m = fmaxf(m, fabsf(s16 ? __fdividef(xv, __half2float(__ushort_as_half(s16[c]))) : xv));
     }
     for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n_scales; k += step)
         d = fmaxf(d, fabsf(__half2float(__ushort_as_half(scales[k]))));
@@ -99,8 +99,8 @@ __global__ void xs_perm_kernel(const uint16_t *__restrict__ x, const uint16_t *_
          q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int64_t m = q / I, c = q % I;
         const int64_t src = (c & ~int64_t(7)) + perm8(static_cast<int>(c & 7));
-        const float v = __fdividef(__uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16),
-                                   __half2float(__ushort_as_half(s16[src])));
+        const float xv = __uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16);
+        const float v = s16 ? __fdividef(xv, __half2float(__ushort_as_half(s16[src]))) : xv;
         xs[q] = __half_as_ushort(__float2half_rn(v * sc));
     }
 }
