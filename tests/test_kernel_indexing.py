@@ -120,9 +120,12 @@ def test_gemv_activation_table_conflict_free(MT):
             assert len(groups) == 8
 
 
+SEARCH_TILE_N, SEARCH_SUB_N = 512, 256     # tokens per unit, per MMA (two halves per unit)
+
+
 def search_units(O, N, G, pairs):
     """Partials the pair search kernel writes: {(g, tb, row): count}."""
-    TILE_O, PAIR_O, TILE_N = 128, 256, 512
+    TILE_O, PAIR_O, TILE_N = 128, 256, SEARCH_TILE_N
     OT = -(-O // PAIR_O)
     TB = -(-N // TILE_N)
     U = OT * TB * G
@@ -152,3 +155,41 @@ def test_search_pairs_write_every_partial_once(O, N, G):
     p = min(U, 74)
     per = [len(range(c, U, p)) for c in range(p)]
     assert max(per) - min(per) <= 1
+
+
+@pytest.mark.parametrize("N", [1, 128, 129, 256, 257, 511, 512, 513, 4096, 65536 + 77])
+def test_search_token_halves_cover_each_token_once(N):
+    """Each unit of 512 tokens runs one or two MMA halves of 256 (two when more
+    than 256 tokens are left); each CTA of the pair stages 128 tokens of a half.
+    Every token below N is staged exactly once; staged rows past N are the
+    zero-filled tail of the last box."""
+    TB = -(-N // SEARCH_TILE_N)
+    seen = {}
+    for tb in range(TB):
+        left = N - tb * SEARCH_TILE_N
+        nsub = 2 if left > SEARCH_SUB_N else 1
+        for h in range(nsub):
+            for rank in (0, 1):
+                y0 = tb * SEARCH_TILE_N + h * SEARCH_SUB_N + rank * SEARCH_SUB_N // 2
+                for t in range(y0, y0 + SEARCH_SUB_N // 2):
+                    if t < N:
+                        seen[t] = seen.get(t, 0) + 1
+                    else:
+                        assert tb == TB - 1
+    assert len(seen) == N and set(seen.values()) == {1}
+
+
+def test_search_tmem_and_shared_memory_plan():
+    """TMEM: the 2 x 256 fp32 accumulator columns fill the 512 columns; the X
+    ring stage (128 tokens x 64 fp16) keeps the 1024-byte alignment the 128-byte
+    swizzle needs; both shared-memory plans (6 X stages, 3 dW stages, 3 or 2
+    input stages) fit 227 KB."""
+    SLAB_K = 64
+    assert 2 * SEARCH_SUB_N <= 512
+    x_stage = (SEARCH_SUB_N // 2) * SLAB_K * 2
+    assert x_stage % 1024 == 0
+    a_stage = 128 * SLAB_K * 2
+    for w_bytes, IS in ((16384, 3), (32768, 2)):
+        in_stage = -(-(w_bytes + 512 + 4096) // 1024) * 1024
+        bars = 2 * 6 + 2 * 3 + 2 * IS + 5
+        assert 1024 + 6 * x_stage + 3 * a_stage + IS * in_stage + bars * 8 + 16 <= 232448

@@ -211,7 +211,7 @@ UNIT_MIXES = [[2, 2, 2], [1], [2, 1, 2, 1], [1, 1, 2], [2] * 5]
 
 @pytest.mark.parametrize("nK", [1, 2, 3])
 @pytest.mark.parametrize("units", UNIT_MIXES)
-@pytest.mark.parametrize("rings", [(6, 3, 3), (6, 3, 2), (2, 1, 1), (4, 2, 2)])
+@pytest.mark.parametrize("rings", [(6, 3, 3), (6, 3, 2), (8, 2, 3), (2, 1, 1), (4, 2, 2)])
 def test_pair_pipeline_protocol(nK, units, rings):
     XS, AS, IS = rings
     for seed in range(8):

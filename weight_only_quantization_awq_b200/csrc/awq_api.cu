@@ -663,10 +663,22 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (M <= 4) {
-        // decode: CUDA-core kernels streaming the packed weights
+        // decode: CUDA-core kernels streaming the packed weights, one launch
         kt_reset(3);
         kt_begin(3, st);
         AWQ_CUDA(awq::launch_w4a16(x, M, in, out, qweight, scales, zeros, s16, group_size, y, st));
+        kt_end(3, st);
+        return AWQ_OK;
+    }
+    if (M <= awq::W4A16_MMA_MAX_M) {
+        // small batches: warp-level tensor-core kernel streaming the packed weights
+        Workspace ws(st);
+        const int64_t wb = awq::w4a16_mma_workspace_bytes(M, in, group_size);
+        if (awq_status_t s = ws.reserve(wb)) return s;
+        char *wsp = ws.take<char>(wb);
+        kt_reset(3);
+        kt_begin(3, st);
+        AWQ_CUDA(awq::launch_w4a16_mma(x, M, in, out, qweight, scales, zeros, s16, group_size, y, wsp, st));
         kt_end(3, st);
         return AWQ_OK;
     }

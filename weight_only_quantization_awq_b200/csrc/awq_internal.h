@@ -25,7 +25,8 @@ constexpr int MAX_GRID = 64;       // grid points per search phase
 // above any legitimate wait in these kernels.
 constexpr long long AWQ_DEFAULT_WAIT_CYCLES = 4000000000LL;
 
-// Search tile shape: 128 output rows x 512 tokens per work unit, K slabs of 64.
+// Search tile shape: 128 output rows per CTA (256 per CTA pair) x 512 tokens per
+// work unit (two MMA halves of 256), K slabs of 64.
 constexpr int TILE_O = 128;
 constexpr int TILE_N = 512;
 constexpr int SUB_N = 256;
@@ -63,7 +64,7 @@ cudaError_t launch_group_params(const void *W, bool w_bf16, int64_t O, int64_t I
 
 // ---- fused search
 // Tensor maps of the kernel's four inputs:
-//   x  : fp16 copy of X [N, I], box 64 x 256, 128B swizzle
+//   x  : fp16 copy of X [N, I], box 64 x 128 (one CTA's half of a 256-token tile), 128B swizzle
 //   w  : W [O, I] (bf16: box 64 x 128; fp32: box 32 x 128), 128B swizzle
 //   sn : scale table [2G, I] fp32, box 64 x 2
 //   qp : group parameters [G * I/gs][O][4] fp32 (3-D), box 4 x 128 rows x groups per slab
@@ -119,6 +120,14 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const uint16_t *scales, const uint32_t *zeros, const uint16_t *s16,
                             int gs, uint16_t *y, const TcPlan &plan, char *workspace,
                             const TcMaps &maps, cudaStream_t st);
+
+// ---- W4A16 apply for decode-sized M (1..16): xs preparation + warp-level MMA kernel
+constexpr int64_t W4A16_MMA_MAX_M = 16;
+int64_t w4a16_mma_workspace_bytes(int64_t M, int64_t I, int gs);
+cudaError_t launch_w4a16_mma(const uint16_t *x, int64_t M, int64_t I, int64_t O,
+                             const uint32_t *qweight, const uint16_t *scales, const uint32_t *zeros,
+                             const uint16_t *s16, int gs, uint16_t *y, char *workspace,
+                             cudaStream_t st);
 
 // ---- W4A16 apply
 // Streaming GEMV for 1 <= M <= 4 (activations staged per CTA; see k_w4a16_stream.cu).

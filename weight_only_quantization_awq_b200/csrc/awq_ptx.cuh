@@ -55,16 +55,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase has not completed is
+// suspended in hardware (issuing nothing) until the phase completes or about
+// `ns` nanoseconds have passed, whichever comes first.
+constexpr uint32_t AWQ_SUSPEND_NS = 1000000;
+
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false if the
 // CTA abort flag is (or becomes) set, or after `limit` SM clock cycles (a
 // kernel argument, AWQ_WAIT_CYCLES by default), in which case it sets the abort
-// flag itself.
+// flag itself.  Each poll suspends the thread for up to AWQ_SUSPEND_NS, so a
+// waiting warp takes no issue slots from the warps doing the work, and the
+// bound is checked between polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
                                           long long limit = AWQ_WAIT_CYCLES) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_for(bar, parity, AWQ_SUSPEND_NS)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > limit) {
             *abort_flag = 1;
@@ -73,29 +92,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// As mbar_wait, but sleeping between polls: for waits that usually last a
-// whole work unit, so the waiting warps do not take issue slots from the rest.
+// The same wait, for waits that usually last a whole work unit.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity,
                                                 volatile int *abort_flag,
                                                 long long limit = AWQ_WAIT_CYCLES) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        __nanosleep(256);
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > limit) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
+    return mbar_wait(bar, parity, abort_flag, limit);
 }
 
 // Same, ignoring the abort flag (used only to drain in-flight copies on exit).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity,
                                                 long long limit = AWQ_WAIT_CYCLES) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_for(bar, parity, AWQ_SUSPEND_NS)) {
         if (clock64() - t0 > limit) return false;
     }
     return true;

@@ -18,7 +18,7 @@
 // and stores half of the X tiles a single-CTA MMA of the same shape would need
 // (the tensor cores of the pair read each other's halves).
 //
-// Warp roles (704 threads per CTA):
+// Warp roles (736 threads per CTA):
 //   warps 0-15  dW producers (16 columns of one row per thread): read one slab's
 //               inputs (W tile, s and -1/s, group parameters) from shared
 //               memory, form dW for the CTA's 128 rows x 64 columns, write it
@@ -28,11 +28,13 @@
 //               (lane = output row), square-and-sum per row, one fp32 partial
 //               per (grid point, token block, row); each 256-column half is
 //               handed back to the MMA as soon as it has been read.
-//   warp 20     TMA: lane 0 streams this CTA's half of the X tiles (128 tokens x
-//               64 channels, fp16 copy of X scaled by a power of two) into the X
-//               ring, counted on the leader's x_full; lane 1 streams each slab's
-//               producer inputs into the (local) input ring.
-//   warp 21     MMA: both CTAs allocate 512 TMEM columns as a pair; in the
+//   warp 20     TMA, one lane: this CTA's half of the X tiles (128 tokens x 64
+//               channels, fp16 copy of X scaled by a power of two) into the X
+//               ring, counted on the leader's x_full.
+//   warp 21     TMA, one lane: each slab's producer inputs into the (local) input
+//               ring.  (The two loaders wait on different barriers, so each has a
+//               warp of its own.)
+//   warp 22     MMA: both CTAs allocate 512 TMEM columns as a pair; in the
 //               leader (rank 0) one thread issues tcgen05.mma.cta_group::2
 //               M=256 N=256 K=16 (two N=256 halves per slab), and
 //               tcgen05.commit with a multicast arrive releases both CTAs' ring
@@ -51,9 +53,10 @@ namespace {
 
 constexpr int NUM_PRODUCER_WARPS = 16;
 constexpr int EPI_WARP0 = 16;                          // warps 16-19: TMEM lane quadrants 0-3
-constexpr int WARP_TMA = 20;
-constexpr int WARP_MMA = 21;
-constexpr int NUM_THREADS = 22 * 32;
+constexpr int WARP_TMA = 20;                           // X tiles
+constexpr int WARP_IN = 21;                            // producer inputs
+constexpr int WARP_MMA = 22;
+constexpr int NUM_THREADS = 23 * 32;
 constexpr int PAIR_O = 2 * TILE_O;                     // output rows per CTA pair
 constexpr int X_HALF = SUB_N / 2;                      // tokens of an N = 256 tile per CTA
 constexpr int X_STAGE_BYTES = X_HALF * SLAB_K * 2;     // 16 KB of fp16 X
@@ -481,10 +484,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp < EPI_WARP0 + 4) {
         epilogue_role(a, OT, U, TB, tmem_base, acc_full, acc_empty, abort_flag);
     } else if (warp == WARP_TMA) {
-        if (lane == 0)
-            x_loader<P::XS>(a, &maps.x, OT, U, x_ring, x_full, x_empty, abort_flag);
-        else if (lane == 1)
-            input_loader<WBF16>(a, maps, OT, U, in_ring, in_full, in_empty, abort_flag);
+        if (lane == 0) x_loader<P::XS>(a, &maps.x, OT, U, x_ring, x_full, x_empty, abort_flag);
+        __syncwarp();
+    } else if (warp == WARP_IN) {
+        if (lane == 0) input_loader<WBF16>(a, maps, OT, U, in_ring, in_full, in_empty, abort_flag);
         __syncwarp();
     } else {
         if (lane == 0 && rank == 0)

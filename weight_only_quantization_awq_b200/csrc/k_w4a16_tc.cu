@@ -5,7 +5,9 @@
 //                   two chosen from max |x / s16| so the largest magnitude lands in
 //                   [2^14, 2^15), with the 8 columns of each packed word stored in
 //                   the order (0,4,1,5,2,6,3,7) (see below); y is scaled back by 2^k.
-//   w4a16_tc_kernel: one CTA per (128-row tile, token tile of <= 256, K split).
+//   w4a16_tc_kernel: one CTA per (128-row tile, token tile of 64, 128 or 256,
+//                   K split); one K split whenever the tiles alone fill half the
+//                   SMs, so most prefill shapes have no split-K partials.
 //     warp 8 (TMA)  streams the packed codes [128 rows x 8 words] and the xs tile
 //                   [N tokens x 64 columns] of each 64-column slab into a ring;
 //     warps 0-7     dequantise: two threads per row (32 columns each); the next
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 uint8_t *dst = in_ring + st * in_stage;
                 const int32_t kb = static_cast<int32_t>(kb0 + i);
                 mbar_arrive_expect_tx(&in_full[st], Q_BYTES + xs_bytes);
-                tma_load_2d(dst, &maps.xs, &in_full[st], kb * SLAB_K, static_cast<int32_t>(mt * TC_TOKENS));
+                tma_load_2d(dst, &maps.xs, &in_full[st], kb * SLAB_K, static_cast<int32_t>(mt * a.n_tile));
                 tma_load_2d(dst + xs_bytes, &maps.q, &in_full[st], kb * 8, static_cast<int32_t>(ot * 128));
 #pragma unroll
                 for (int s = 0; s < RS; ++s)
@@ -295,7 +297,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         named_bar_sync(1, 128);
         const bool got = ok && nslab > 0 && mbar_wait_sleep(acc_full, 0, abort_flag);
         tc_fence_after();
-        const int64_t m0 = mt * TC_TOKENS;
+        const int64_t m0 = mt * a.n_tile;
         const int mcount = static_cast<int>(a.M - m0 < a.n_tile ? a.M - m0 : a.n_tile);
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         // y = accumulator * 2^kx * 2^kd, two normal factors (their product can be subnormal)
@@ -354,21 +356,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
 TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     TcPlan p;
-    const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
+    const int64_t OT = (O + 127) / 128;
     const int64_t nK = I / SLAB_K;
-    // wide token tiles: about one CTA per SM (the split-K adds grow with the splits);
-    // narrow ones: about two per SM, for latency hiding
-    const int64_t target = M >= 128 ? num_sms : 2 * num_sms;
-    int64_t splits = target / (OT * MT);          // at most one wave
-    if (splits < 1) splits = 1;
-    if (splits > nK) splits = nK;
-    const int64_t spl = (nK + splits - 1) / splits;
-    splits = (nK + spl - 1) / spl;
-    p.splits = static_cast<int>(splits);
-    p.slabs_per_split = static_cast<int>(spl);
-    p.n_tile = static_cast<int>(M >= TC_TOKENS ? TC_TOKENS : (M + 15) / 16 * 16);
+    // One K split when (128-row tile, token tile) pairs alone fill at least half
+    // of the SMs: no split-K partial sums at all.  Among token tiles of 256, 128
+    // and 64 pick the fewest waves x tile width (a 64-token tile runs the MMA at
+    // about 2/3 of the wider tiles' rate: its A tile is re-read per 64 tokens).
+    double best = 0.0;
+    int best_n = 0;
+    for (int n : {256, 128, 64}) {
+        if (n > 64 && M <= n / 2) continue;                  // tile mostly empty
+        const int64_t tiles = OT * ((M + n - 1) / n);
+        if (tiles * 2 < num_sms) continue;
+        const int64_t waves = (tiles + num_sms - 1) / num_sms;
+        const double cost = static_cast<double>(waves) * n * (n == 64 ? 1.5 : 1.0);
+        if (best_n == 0 || cost < best) {
+            best = cost;
+            best_n = n;
+        }
+    }
+    if (best_n > 0) {
+        p.n_tile = best_n < M ? best_n : static_cast<int>((M + 15) / 16 * 16);
+        p.splits = 1;
+        p.slabs_per_split = static_cast<int>(nK);
+    } else {
+        // Narrow or short layers: split K to fill the GPU; the partials meet in an
+        // fp32 tile.  Wide token tiles: about one CTA per SM (the split-K adds grow
+        // with the splits); narrow ones: about two per SM, for latency hiding.
+        p.n_tile = static_cast<int>(M >= TC_TOKENS ? TC_TOKENS : (M + 15) / 16 * 16);
+        const int64_t MT = (M + p.n_tile - 1) / p.n_tile;
+        const int64_t target = M >= 128 ? num_sms : 2 * num_sms;
+        int64_t splits = target / (OT * MT);          // at most one wave
+        if (splits < 1) splits = 1;
+        if (splits > nK) splits = nK;
+        const int64_t spl = (nK + splits - 1) / splits;
+        splits = (nK + spl - 1) / spl;
+        p.splits = static_cast<int>(splits);
+        p.slabs_per_split = static_cast<int>(spl);
+    }
+    const int64_t MT = (M + p.n_tile - 1) / p.n_tile;
     p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
-    p.part_bytes = splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
+    p.part_bytes = p.splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
     p.counter_bytes = (OT * MT * 4 + 16 + 255) / 256 * 256;   // 4 scale words, tile counters
     return p;
 }
@@ -377,7 +405,7 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const uint16_t *scales, const uint32_t *zeros, const uint16_t *s16,
                             int gs, uint16_t *y, const TcPlan &plan, char *workspace,
                             const TcMaps &maps, cudaStream_t st) {
-    const int64_t OT = (O + 127) / 128, MT = (M + TC_TOKENS - 1) / TC_TOKENS;
+    const int64_t OT = (O + 127) / 128, MT = (M + plan.n_tile - 1) / plan.n_tile;
     uint16_t *xs = reinterpret_cast<uint16_t *>(workspace);
     float *acc32 = plan.splits > 1 ? reinterpret_cast<float *>(workspace + plan.xs_bytes) : nullptr;
     unsigned *words = reinterpret_cast<unsigned *>(workspace + plan.xs_bytes + plan.part_bytes);
