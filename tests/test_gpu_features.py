@@ -49,10 +49,14 @@ def u16(t):
 
 
 def check_choice(idx_gpu, idx_ref, loss_ref):
-    if idx_gpu == idx_ref:
-        return
-    gap = abs(loss_ref[idx_gpu] - loss_ref[idx_ref])
-    assert gap <= TIE_RTOL * loss_ref[idx_ref], (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
+    """Exact unless the oracle's best loss has near-ties within 2 x LOSS_RTOL;
+    then any index of that set (see test_gpu_parity.check_choice)."""
+    loss_ref = np.asarray(loss_ref, np.float64)
+    near = np.abs(loss_ref - loss_ref[idx_ref]) <= TIE_RTOL * loss_ref[idx_ref]
+    if near.sum() == 1:
+        assert idx_gpu == idx_ref, (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
+    else:
+        assert near[idx_gpu], (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
 
 
 def check_pack(got, ref, qt):
@@ -255,3 +259,28 @@ def test_group_clip_against_oracle(awq, O, I, N, gs, qt, wbit):
     p = awq.awq_pack_quant(Wd, sXd, alpha, 1.0, gs, qt, w_bit=wbit, clip_idx=got["clip_idx"],
                            clip_grid=CLIP_GRID, scales_f32=True)
     check_pack(p, oracle.pack_int4(W, sX, alpha, 1.0, gs, qt, w_bit=wbit, clip_g=CLIP_GRID[ig]), qt)
+
+
+# ------------------------------------------------------------------ several linears per launch
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_linear_batch_matches_single_calls(awq, M):
+    """The decoder block's seven linear shapes (q, k, v, o 4096x4096; gate, up
+    11008x4096; down 4096x11008, scaled down 8x in their row counts) in one
+    call: every output bit-identical to the single-linear call, which the apply
+    parity tests check against the oracle; one of them is checked here too."""
+    shapes = [(512, 512), (512, 512), (512, 512), (512, 512), (1376, 512), (1376, 512), (512, 1408)]
+    gs = 128
+    layers, refs = [], []
+    for k, (o, i) in enumerate(shapes):
+        W, X = small_layer(o, i, 64, seed=200 + k)
+        pk = oracle.pack_int4(W, oracle.act_stats(X), 0.5, 1.0, gs, oracle.ASYM)
+        x = apply_activations(M, i, seed=k)
+        layers.append((dev(x), dev(pk["qweight"]), dev(pk["scales"]).view(torch.float16),
+                       dev(pk["zeros"]), dev(pk["s16"]).view(torch.float16)))
+        refs.append((x, pk))
+    ys = awq.awq_linear_w4a16_batch(layers, gs)
+    for (xd, q, sc, z, s16), y in zip(layers, ys):
+        y1 = awq.awq_linear_w4a16(xd, q, sc, z, s16, gs)
+        assert torch.equal(y, y1)
+    x, pk = refs[6]
+    check_apply(ys[6], oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], gs))

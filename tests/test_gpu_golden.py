@@ -51,7 +51,11 @@ def dev(a):
 
 
 def near_tie(idx_gpu, idx_ref, loss_ref):
-    return idx_gpu == idx_ref or abs(loss_ref[idx_gpu] - loss_ref[idx_ref]) <= TIE_RTOL * loss_ref[idx_ref]
+    """Exact unless the oracle's best loss has near-ties within 2 x LOSS_RTOL (the
+    most two losses each within LOSS_RTOL can swap by); then any of that set."""
+    loss_ref = np.asarray(loss_ref, np.float64)
+    near = np.abs(loss_ref - loss_ref[idx_ref]) <= TIE_RTOL * loss_ref[idx_ref]
+    return idx_gpu == idx_ref if near.sum() == 1 else bool(near[idx_gpu])
 
 
 @pytest.mark.parametrize("wid,layer", LAYERS)

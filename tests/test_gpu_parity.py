@@ -47,10 +47,16 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 
 def check_choice(idx_gpu, idx_ref, loss_ref):
-    if idx_gpu == idx_ref:
-        return
-    gap = abs(loss_ref[idx_gpu] - loss_ref[idx_ref])
-    assert gap <= TIE_RTOL * loss_ref[idx_ref], (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
+    """The selected index equals the oracle's whenever the oracle's best loss is
+    separated from every other by more than 2 x LOSS_RTOL (the most two losses
+    each within LOSS_RTOL can swap by); otherwise any index of the oracle's
+    near-tie set is a correct minimiser."""
+    loss_ref = np.asarray(loss_ref, np.float64)
+    near = np.abs(loss_ref - loss_ref[idx_ref]) <= TIE_RTOL * loss_ref[idx_ref]
+    if near.sum() == 1:
+        assert idx_gpu == idx_ref, (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
+    else:
+        assert near[idx_gpu], (idx_gpu, idx_ref, loss_ref[idx_gpu], loss_ref[idx_ref])
 
 
 # --------------------------------------------------------------------- stats
