@@ -348,8 +348,17 @@ def run_ours(args, rank, world, local_rank):
 
     block_apply = measure_block_apply(dev)
     extra_search = measure_search_only(2, awq, dev) if wid != 2 else None
+    block_search = measure_block_search(awq, dev) if args.block_search else None
 
     pk_ = peaks()
+    # A kernel timed inside a timed region of a second or more runs under the
+    # power cap: its roofline is the sustained GEMM figure; a short burst, the burst one.
+    if ms >= 1000.0:
+        peak, peak_kind = pk_["bf16_tflops_sustained"], "sustained"
+        peak_why = f"the search kernel runs back to back for {ms / 1e3:.1f} s"
+    else:
+        peak, peak_kind = pk_["bf16_tflops"], "burst"
+        peak_why = f"timed region {ms:.0f} ms"
     search_kernel_ms = statistics.mean(search_ms) if search_ms else None
     achieved = flops_step / (search_kernel_ms * 1e-3) / 1e12 if search_kernel_ms else None
     sha = source_sha(os.path.join(ROOT, "weight_only_quantization_awq_b200", "csrc", "k_search.cu"))
@@ -376,9 +385,12 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "roofline": {"bound": "tensor", "kernel": "search_kernel",
                      "achieved": round(achieved, 2) if achieved else None,
-                     "peak": pk_["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": round(achieved / pk_["bf16_tflops"], 4) if achieved else None,
-                     "peak_source": pk_["source"] + " burst bf16",
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4) if achieved else None,
+                     "peak_source": f"{pk_['source']} {peak_kind} bf16 ({peak_why})",
+                     "frac_burst": round(achieved / pk_["bf16_tflops"], 4) if achieved else None,
+                     "frac_sustained": (round(achieved / pk_["bf16_tflops_sustained"], 4)
+                                        if achieved else None),
                      "kernel_ms": round(search_kernel_ms, 4) if search_kernel_ms else None,
                      "algorithmic_flops": flops_step,
                      "traffic": traffic},
@@ -389,9 +401,15 @@ def run_ours(args, rank, world, local_rank):
                   "frac_hbm": round(apply_bytes / (apply_us * 1e-6) / 1e9 / pk_["hbm_gbs"], 4),
                   "bytes": apply_bytes,
                   "timing": f"CUDA graph of {reps * n_copies} launches over {n_copies} packed copies"},
-        "w4a16_block": {str(m): {**v, "frac_hbm": round(v["gb_per_s"] / pk_["hbm_gbs"], 4)}
+        "w4a16_block": {str(m): {**v, "frac_hbm": round(v["gb_per_s"] / pk_["hbm_gbs"], 4),
+                                 **({"batched": {**v["batched"], "frac_hbm": round(
+                                     v["batched"]["gb_per_s"] / pk_["hbm_gbs"], 4)}}
+                                    if "batched" in v else {})}
                         for m, v in block_apply.items()},
     }
+    if block_search is not None:
+        block_search["frac_sustained"] = round(block_search["tflops"] / pk_["bf16_tflops_sustained"], 4)
+        out["search_block"] = block_search
     if extra_search is not None:
         extra_search["frac"] = round(extra_search["tflops"] / pk_["bf16_tflops"], 4)
         out["search_" + extra_search["workload"]] = extra_search
@@ -425,6 +443,38 @@ def graph_time_us(fn, reps):
     torch.cuda.synchronize()
     del g
     return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def measure_block_search(awq, dev, reps=2):
+    """The Llama-7B block's searches (workload 5: qkv 12288x4096, o 4096x4096,
+    gate||up 22016x4096, down 4096x11008; 16384 tokens each, asymmetric INT4
+    g128, 20 alphas then 11 clip ratios at alpha*): search-kernel device time
+    per block (library CUDA events, both phases), mean of `reps` passes."""
+    import torch
+    import synthetic
+    from synthetic import ALPHA_GRID, CLIP_GRID
+    wl = synthetic.workload(5)
+    alphas, clips = [float(a) for a in ALPHA_GRID], [float(c) for c in CLIP_GRID]
+    awq.set_kernel_timing(True)
+    per_layer, flops = {}, 0.0
+    for L in wl.layers:
+        Wd = _bf16_dev(synthetic.layer_weights(5, L.name), dev)
+        Xd = _bf16_dev(synthetic.layer_activations(5, L.name), dev)
+        sX = awq.awq_act_stats(Xd)
+        awq.awq_search_layer(Wd, Xd, sX, GROUP, 4, "asym", alphas, clip=clips)   # warm-up
+        ms = []
+        for _ in range(reps):
+            awq.awq_search_layer(Wd, Xd, sX, GROUP, 4, "asym", alphas, clip=clips)
+            ms.append(awq.last_kernel_ms(awq.KT_SEARCH))
+        per_layer[L.name] = round(statistics.mean(ms), 3)
+        flops += (len(alphas) + len(clips)) * 2.0 * wl.tokens * L.inp * L.out
+        del Wd, Xd
+        torch.cuda.empty_cache()
+    awq.set_kernel_timing(False)
+    total = sum(per_layer.values())
+    return {"workload": wl.name, "kernel_ms": round(total, 3), "per_layer_ms": per_layer,
+            "tflops": round(flops / (total * 1e-3) / 1e12, 2), "algorithmic_flops": flops,
+            "timing": f"library CUDA events around the search kernel (alpha and clip phases), mean of {reps}"}
 
 
 def measure_search_only(wid, awq, dev, reps=6):
@@ -489,12 +539,24 @@ def measure_block_apply(dev, ms=(1, 16, 256), copies=2, reps=4):
                     awq.awq_linear_w4a16(xs[i], p["qweight"], p["scales"], p["zeros"], p["s16"],
                                          GROUP, out=ys[k])
 
+        def run_batched():
+            for layer in packs:
+                awq.awq_linear_w4a16_batch(
+                    [(xs[i], p["qweight"], p["scales"], p["zeros"], p["s16"]) for p, o, i in layer],
+                    GROUP, outs=ys)
+
         us = graph_time_us(run_all, reps) / copies
         byts = sum(p["qweight"].numel() * 4 + p["scales"].numel() * 2 + p["zeros"].numel() * 4 +
                    p["s16"].numel() * 2 + m * i * 2 + m * o * 2 for p, o, i in packs[0])
         flops = sum(2.0 * m * o * i for _, o, i in BLOCK_LINEARS)
         out[m] = {"us_per_block": round(us, 2), "gb_per_s": round(byts / (us * 1e-6) / 1e9, 1),
-                  "tflops": round(flops / (us * 1e-6) / 1e12, 2), "bytes": byts}
+                  "tflops": round(flops / (us * 1e-6) / 1e12, 2), "bytes": byts,
+                  "timing": f"one launch per linear, CUDA graph of {reps} passes over {copies} packed copies"}
+        if m <= 8:
+            ub = graph_time_us(run_batched, reps) / copies
+            out[m]["batched"] = {"us_per_block": round(ub, 2),
+                                 "gb_per_s": round(byts / (ub * 1e-6) / 1e9, 1),
+                                 "timing": "awq_linear_w4a16_batch: the seven linears in one launch"}
     return out
 
 
@@ -584,6 +646,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, choices=sorted(BENCH_WORKLOADS), default=4)
+    ap.add_argument("--block-search", dest="block_search", action=argparse.BooleanOptionalAction,
+                    default=True, help="also time the Llama-7B block's four joint layers' searches")
     args = ap.parse_args()
     if args.steps is None:
         args.steps = BENCH_WORKLOADS[args.workload]["steps"]

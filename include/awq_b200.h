@@ -211,20 +211,51 @@ awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in,
  * operator that produces x, see awq_fold_scale) and is used as is.
  * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.  in <= 49152.
  * Storage arguments as produced by awq_pack_int4.  Asynchronous.
- * Precision: x / s16 is rounded to fp16 after a power-of-two scale (2^-11
- * relative); for M >= 5 (tensor cores) (code - z) * scale is also rounded to
- * fp16 once.  M <= 4 runs on the CUDA cores and needs no workspace.
- * Ordering: the M <= 4 kernel is launched with programmatic stream
- * serialisation, so its blocks may start while the preceding kernel on
- * `stream` is still running; until that kernel has completed they only ask L2
- * to prefetch qweight, scales, zeros, s16 and x (a hint that reads nothing
- * into the SM), and every read of an argument, and the write of y, happens
- * after it.
+ * Kernels by M: 1..4 a CUDA-core kernel streaming the packed weights (no
+ * workspace); 5..16 warp-level tensor-core MMA on the unpacked codes (an x / s
+ * workspace); 17 and more tcgen05 tensor-core tiles.
+ * Precision: x / s16 is rounded to fp16 after a power-of-two scale per
+ * (token, group) (2^-11 relative); for M >= 17 (code - z) * scale is also
+ * rounded to fp16 once.  Accumulation in fp32.
+ * Ordering: the kernels are launched with programmatic stream serialisation,
+ * so their blocks may start while the preceding kernel on `stream` is still
+ * running; until that kernel has completed they only ask L2 to prefetch
+ * their weights (a hint that reads nothing into the SM), and every read of an
+ * argument, and the write of y, happens after it.
  */
 awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t out,
                               const uint32_t *qweight, const uint16_t *scales,
                               const uint32_t *zeros, const uint16_t *s16,
                               int group_size, uint16_t *y, void *stream);
+
+/*
+ * awq_linear_w4a16_batch — awq_linear_w4a16 on up to AWQ_MAX_BATCH_LINEARS
+ * independent linears at once (e.g. the projections of a decoder block that
+ * read the same or different inputs): y_k = (x_k / s16_k) * dequant(W_k)^T for
+ * every descriptor k, all at the same M and group_size, with zero points given
+ * for every linear or for none ([AWQ-guide] 三, QuantLinear.forward).
+ * For M <= 8, when the staged activations of the widest linear and a ring of
+ * weight tiles fit one SM's shared memory (M <= 6 at in = 11008, M <= 8 at
+ * in = 4096), this is one persistent launch, one block per SM: the 16-row
+ * tiles of all linears are dealt out in contiguous, byte-balanced ranges, so
+ * the layers share one ramp-up of the memory system; otherwise the linears run
+ * one after the other through awq_linear_w4a16.  Each output is bit-identical
+ * to the same call with that linear alone.  Precision as awq_linear_w4a16.
+ * The outputs must not overlap each other or any input.  Asynchronous.
+ */
+#define AWQ_MAX_BATCH_LINEARS 8
+typedef struct {
+    const uint16_t *x;          /* [M, in] bf16 device */
+    int64_t in, out;
+    const uint32_t *qweight;    /* [out][in/8] u32 device (awq_pack_int4 layout) */
+    const uint16_t *scales;     /* [out][in/group_size] fp16 bits device */
+    const uint32_t *zeros;      /* [out][ceil(in/group_size/8)] u32 device, or NULL (symmetric) */
+    const uint16_t *s16;        /* [in] fp16 bits device, or NULL (x already divided by s) */
+    uint16_t *y;                /* [M, out] bf16 device, written */
+} awq_linear_desc_t;
+
+awq_status_t awq_linear_w4a16_batch(const awq_linear_desc_t *descs, int n, int64_t M,
+                                    int group_size, void *stream);
 
 /*
  * awq_fold_scale — fold the division by s into the operator that produces

@@ -175,3 +175,25 @@ def test_linear_accepts_missing_scale_vector_on_host():
     f = lib.awq_linear_w4a16
     st = f(FAKE, 1, 4096, 4096, FAKE, FAKE, NULL, NULL, 128, FAKE, NULL)
     assert st not in (ARG, ALIGN, UNSUP)
+
+
+def test_linear_batch_rejects_on_host():
+    from weight_only_quantization_awq_b200 import _LinearDesc
+    f = lib.awq_linear_w4a16_batch
+
+    def descs(*mods):
+        d = (_LinearDesc * len(mods))()
+        for k, m in enumerate(mods):
+            v = dict(x=FAKE, in_=4096, out=4096, qweight=FAKE, scales=FAKE, zeros=FAKE, s16=FAKE, y=FAKE)
+            v.update(m)
+            d[k] = _LinearDesc(**v)
+        return ctypes.cast(d, ctypes.c_void_p)
+    assert f(NULL, 1, 1, 128, NULL) == ARG
+    assert f(descs({}), 0, 1, 128, NULL) == ARG
+    assert f(descs(*([{}] * 9)), 9, 1, 128, NULL) == ARG
+    assert f(descs({}), 1, 0, 128, NULL) == ARG
+    assert f(descs({}), 1, 1, 96, NULL) == UNSUP
+    assert f(descs({}, {"zeros": None}), 2, 1, 128, NULL) == ARG      # zero points for some only
+    assert f(descs({}, {"y": None}), 2, 1, 128, NULL) == ARG
+    assert f(descs({}, {"in_": 100}), 2, 1, 128, NULL) == UNSUP
+    assert f(descs({}, {"x": FAKE + 2}), 2, 1, 128, NULL) == ALIGN

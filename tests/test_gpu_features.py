@@ -263,11 +263,12 @@ def test_group_clip_against_oracle(awq, O, I, N, gs, qt, wbit):
 
 # ------------------------------------------------------------------ several linears per launch
 @pytest.mark.parametrize("M", [1, 3, 8])
-def test_linear_batch_matches_single_calls(awq, M):
+def test_linear_batch_block_shapes_against_oracle(awq, M):
     """The decoder block's seven linear shapes (q, k, v, o 4096x4096; gate, up
     11008x4096; down 4096x11008, scaled down 8x in their row counts) in one
-    call: every output bit-identical to the single-linear call, which the apply
-    parity tests check against the oracle; one of them is checked here too."""
+    call: every output within the apply tolerance of the oracle, and each equal
+    to what the same call gives for that linear alone (the tiles a linear
+    contributes do not depend on the other linears of the launch)."""
     shapes = [(512, 512), (512, 512), (512, 512), (512, 512), (1376, 512), (1376, 512), (512, 1408)]
     gs = 128
     layers, refs = [], []
@@ -277,10 +278,35 @@ def test_linear_batch_matches_single_calls(awq, M):
         x = apply_activations(M, i, seed=k)
         layers.append((dev(x), dev(pk["qweight"]), dev(pk["scales"]).view(torch.float16),
                        dev(pk["zeros"]), dev(pk["s16"]).view(torch.float16)))
-        refs.append((x, pk))
+        refs.append(oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], gs))
     ys = awq.awq_linear_w4a16_batch(layers, gs)
-    for (xd, q, sc, z, s16), y in zip(layers, ys):
-        y1 = awq.awq_linear_w4a16(xd, q, sc, z, s16, gs)
+    for layer, y, y_ref in zip(layers, ys, refs):
+        check_apply(y, y_ref)
+        (y1,) = awq.awq_linear_w4a16_batch([layer], gs)
         assert torch.equal(y, y1)
-    x, pk = refs[6]
-    check_apply(ys[6], oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], gs))
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8])
+@pytest.mark.parametrize("gs,qt,with_s", [(64, oracle.ASYM, True), (128, oracle.SYM, False),
+                                           (32, oracle.ASYM, True)])
+def test_linear_batch_ragged_against_oracle(awq, M, gs, qt, with_s):
+    """One launch over linears with ragged shapes, each output checked against
+    the oracle: a last row tile of 5 or 8 rows whose scales are not 16-byte
+    sized, an odd group count per row, an input width ending 64 columns into a
+    1024-column stage, a single 16 x 64 tile, and more tiles in all than there
+    are SMs, so CTAs cross from one linear into the next."""
+    shapes = [(37, 1088), (512, 2112), (1000, 640), (16, 64), (3000, 1024), (200, 384)]
+    shapes = [(o, i) for o, i in shapes if i % gs == 0]
+    layers, refs = [], []
+    for k, (o, i) in enumerate(shapes):
+        W, X = small_layer(o, i, 32, seed=300 + k)
+        pk = oracle.pack_int4(W, oracle.act_stats(X), 0.5, 1.0, gs, qt)
+        x = apply_activations(M, i, seed=40 + k)
+        s16 = pk["s16"] if with_s else None
+        layers.append((dev(x), dev(pk["qweight"]), dev(pk["scales"]).view(torch.float16),
+                       dev(pk["zeros"]) if pk["zeros"] is not None else None,
+                       dev(s16).view(torch.float16) if s16 is not None else None))
+        refs.append(oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], s16, gs))
+    ys = awq.awq_linear_w4a16_batch(layers, gs)
+    for y, y_ref in zip(ys, refs):
+        check_apply(y, y_ref)

@@ -9,6 +9,12 @@ and check the invariants the kernels rely on:
   pointer steps.  Every (row, 32-column chunk) must be loaded exactly once, by
   an in-bounds address equal to the direct index, and the lane's zero nibble
   must be the group's.
+* W4A16 batched decode (csrc/k_w4a16_dec.cu): units of 16 rows x 4096 columns
+  over a list of linears; CTA c owns the 16-row tiles whose first unit is in
+  [c U / P, (c + 1) U / P).  Every tile must be owned by exactly one CTA, the
+  tiles a CTA walks must be consecutive, and no CTA may stream much more than
+  its share; the staged activations must land in distinct, in-bounds 16-byte
+  slots whose four fragment-thread reads of a token are one contiguous span.
 * Fused search (csrc/k_search.cu): CTA pairs deal work units (grid point, 256-row
   pair tile, 512-token block) round-robin; every (grid point, row, token block)
   partial must be written exactly once.
@@ -193,3 +199,107 @@ def test_search_tmem_and_shared_memory_plan():
         in_stage = -(-(w_bytes + 512 + 4096) // 1024) * 1024
         bars = 2 * 6 + 2 * 3 + 2 * IS + 5
         assert 1024 + 6 * x_stage + 3 * a_stage + IS * in_stage + bars * 8 + 16 <= 232448
+
+
+# ---- batched decode: partition of tiles over CTAs, staged activation slots
+DEC_KC = 4096
+
+
+def dec_units(linears):
+    """ucum and stages-per-tile of a list of (out, in) linears."""
+    ucum, spt = [0], []
+    for O, I in linears:
+        s = -(-I // DEC_KC)
+        spt.append(s)
+        ucum.append(ucum[-1] + -(-O // 16) * s)
+    return ucum, spt
+
+
+def dec_cta_tiles(ucum, spt, u0, u1):
+    """The kernel's dec_first_tile / dec_next_tile walk, restated."""
+    n = len(spt)
+    l = 0
+    while l + 1 < n and u0 >= ucum[l + 1]:
+        l += 1
+    t = (u0 - ucum[l] + spt[l] - 1) // spt[l]
+    a = ucum[l] + t * spt[l]
+    if a >= ucum[l + 1]:
+        if l + 1 >= n:
+            return []
+        l, t, a = l + 1, 0, ucum[l + 1]
+    out = []
+    while a < u1:
+        out.append((l, t, a))
+        a += spt[l]
+        t += 1
+        if a >= ucum[l + 1]:
+            if l + 1 >= n:
+                break
+            l, t, a = l + 1, 0, ucum[l + 1]
+    return out
+
+
+BLOCK7 = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
+
+
+@pytest.mark.parametrize("linears,sms", [
+    (BLOCK7, 148), ([(4096, 4096)], 148), ([(12288, 4096), (4096, 4096), (22016, 4096), (4096, 11008)], 148),
+    ([(17, 64), (5, 1088), (100, 2048)], 148), ([(16, 64)], 148), ([(4100, 4160)], 7),
+    ([(1, 64)] * 8, 3), ([(33, 3072), (2000, 1024)], 148)])
+def test_decode_tiles_owned_once_and_balanced(linears, sms):
+    ucum, spt = dec_units(linears)
+    U = ucum[-1]
+    tiles = sum(-(-O // 16) for O, _ in linears)
+    P = min(sms, tiles)
+    owner = {}
+    biggest = max(spt)
+    for c in range(P):
+        u0, u1 = c * U // P, (c + 1) * U // P
+        walk = dec_cta_tiles(ucum, spt, u0, u1)
+        for k, (l, t, a) in enumerate(walk):
+            assert 0 <= t < -(-linears[l][0] // 16)
+            assert a == ucum[l] + t * spt[l] and u0 <= a < u1
+            assert (l, t) not in owner
+            owner[(l, t)] = c
+            if k:
+                pl, pt, _ = walk[k - 1]
+                assert (l, t) == (pl, pt + 1) or (l == pl + 1 and t == 0)
+        units = sum(spt[l] for l, _, _ in walk)
+        # a CTA streams at most its share plus one tile
+        assert units <= U / P + biggest
+    assert len(owner) == tiles
+
+
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_decode_staged_slots_distinct_and_contiguous(gs):
+    """Word wg of a group (thread j = wg // NW, its kk = wg % NW) goes to slot
+    4 kk + j: a bijection onto the group's slots, and thread j's kk-th read
+    (slot 4 kk + j) for j = 0..3 covers 4 consecutive slots."""
+    WPG, NW = gs // 8, gs // 32
+    slots = [(wg % NW) * 4 + wg // NW for wg in range(WPG)]
+    assert sorted(slots) == list(range(WPG))
+    for kk in range(NW):
+        got = [slots[NW * j + kk] for j in range(4)]
+        assert got == [4 * kk + j for j in range(4)]
+
+
+def test_decode_shared_memory_plan_fits():
+    """The Llama-7B block linears at M = 1 take the 2-buffer plan with four
+    33 KB stages, at M = 2 a 2-buffer plan still; at M = 8 the 4096-wide linears
+    still fit; an 11008-wide linear at M = 8 does not."""
+    def smem(M, linears, gs, zeros, st, hb, xb):
+        hdr = max(32 * (I // gs) + (64 * -(-(I // gs) // 8) if zeros else 0) for _, I in linears)
+        xbuf = max(M * (I + 32) * 2 + -(-(M * (I // gs) * 8) // 16) * 16 for _, I in linears)
+        hdr, xbuf = -(-hdr // 128) * 128, -(-xbuf // 128) * 128
+        return st * 16 * 2112 + hb * hdr + xb * xbuf + 2 * 8 * 16 * 8 * 4 + (2 * st + 2 * hb + 2 * xb) * 8 + 16
+
+    def plan(M, linears):
+        for o in ((4, 3, 2), (3, 3, 2), (4, 3, 1), (3, 2, 1), (2, 2, 1)):
+            if smem(M, linears, 128, True, *o) <= 227 * 1024:
+                return o
+        return None
+
+    assert plan(1, BLOCK7) == (4, 3, 2)
+    assert plan(2, BLOCK7) is not None and plan(2, BLOCK7)[2] == 2
+    assert plan(8, [(4096, 4096)]) is not None
+    assert plan(8, BLOCK7) is None

@@ -69,6 +69,8 @@ def _load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.awq_search_points.argtypes = [P, I, L, L, P, I, L, P, I, I, I, P, P, I, P, P, P, P]
     lib.awq_pack_quant.restype = I
     lib.awq_pack_quant.argtypes = [P, I, L, L, P, D, D, P, P, I, I, I, I, P, P, P, P, P, P]
+    lib.awq_linear_w4a16_batch.restype = I
+    lib.awq_linear_w4a16_batch.argtypes = [P, I, L, I, P]
     lib.awq_group_clip.restype = I
     lib.awq_group_clip.argtypes = [P, I, L, L, P, I, L, P, D, I, I, I, P, I, P, P, P]
     lib.awq_fold_scale.restype = I
@@ -87,7 +89,8 @@ lib = _load_library()
 EXPORTS = ("awq_version", "awq_status_string", "awq_last_error", "awq_act_stats",
            "awq_search_layer", "awq_search_points", "awq_group_clip", "awq_pack_int4",
            "awq_pack_quant",
-           "awq_linear_w4a16", "awq_fold_scale", "awq_wait_selftest", "awq_set_kernel_timing",
+           "awq_linear_w4a16", "awq_linear_w4a16_batch", "awq_fold_scale", "awq_wait_selftest",
+           "awq_set_kernel_timing",
            "awq_last_kernel_ms", "awq_act_stats_noalloc")
 
 MAX_POINTS = 4096
@@ -358,3 +361,44 @@ def awq_linear_w4a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tenso
         s16.data_ptr() if s16 is not None else None, group_size, out.data_ptr(), _stream(x))
     _check("awq_linear_w4a16", st)
     return out
+
+
+class _LinearDesc(ctypes.Structure):
+    """awq_linear_desc_t of the C ABI."""
+    _fields_ = [("x", ctypes.c_void_p), ("in_", ctypes.c_int64), ("out", ctypes.c_int64),
+                ("qweight", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p), ("s16", ctypes.c_void_p), ("y", ctypes.c_void_p)]
+
+
+MAX_BATCH_LINEARS = 8
+
+
+def awq_linear_w4a16_batch(layers, group_size: int = 128, outs=None):
+    """Several independent W4A16 linears at the same M in one call (one kernel
+    launch for M <= 8).  `layers`: list of (x, qweight, scales, zeros, s16); returns
+    the list of y [M, out] bf16 (or fills `outs`)."""
+    if not 1 <= len(layers) <= MAX_BATCH_LINEARS:
+        raise ValueError(f"1..{MAX_BATCH_LINEARS} linears per call")
+    M = layers[0][0].shape[0]
+    descs = (_LinearDesc * len(layers))()
+    ys = []
+    for k, (x, qweight, scales, zeros, s16) in enumerate(layers):
+        _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales")
+        if x.dtype != torch.bfloat16 or x.shape[0] != M:
+            raise ValueError("every x must be bfloat16 with the same number of tokens")
+        if zeros is not None:
+            _dev(zeros, "zeros")
+        if s16 is not None:
+            _dev(s16, "s16")
+        out_f = qweight.shape[0]
+        y = outs[k] if outs is not None else torch.empty((M, out_f), dtype=torch.bfloat16,
+                                                          device=x.device)
+        _out(y, "y", x, torch.bfloat16, M * out_f)
+        ys.append(y)
+        descs[k] = _LinearDesc(x.data_ptr(), x.shape[1], out_f, qweight.data_ptr(),
+                               scales.data_ptr(), zeros.data_ptr() if zeros is not None else None,
+                               s16.data_ptr() if s16 is not None else None, y.data_ptr())
+    _check("awq_linear_w4a16_batch",
+           lib.awq_linear_w4a16_batch(ctypes.cast(descs, ctypes.c_void_p), len(layers), M,
+                                      group_size, _stream(layers[0][0])))
+    return ys

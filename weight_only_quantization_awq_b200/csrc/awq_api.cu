@@ -607,6 +607,51 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, 
                           quant, qweight, scales, zeros, s16, scales_f32, stream);
 }
 
+awq_status_t awq_linear_w4a16_batch(const awq_linear_desc_t *descs, int n, int64_t M,
+                                    int group_size, void *stream) {
+    g_last_error.clear();
+    if (!descs) return fail(AWQ_ERR_ARG, "NULL descriptor list");
+    if (n < 1 || n > AWQ_MAX_BATCH_LINEARS) return fail(AWQ_ERR_ARG, "n=%d not in [1, %d]", n, AWQ_MAX_BATCH_LINEARS);
+    if (M < 1) return fail(AWQ_ERR_ARG, "bad M");
+    if (group_size != 32 && group_size != 64 && group_size != 128)
+        return fail(AWQ_ERR_UNSUPPORTED, "group_size %d not in {32, 64, 128}", group_size);
+    const bool zeros = descs[0].zeros != nullptr;
+    awq::DecBatch b{};
+    b.n = n;
+    for (int k = 0; k < n; ++k) {
+        const awq_linear_desc_t &d = descs[k];
+        if (!d.x || !d.qweight || !d.scales || !d.y) return fail(AWQ_ERR_ARG, "linear %d: NULL pointer", k);
+        if (d.in < 1 || d.out < 1) return fail(AWQ_ERR_ARG, "linear %d: bad shape", k);
+        if ((d.zeros != nullptr) != zeros)
+            return fail(AWQ_ERR_ARG, "linear %d: zero points must be given for all linears or for none", k);
+        if (d.in % 64 != 0 || d.in % group_size != 0 || d.in > 49152)
+            return fail(AWQ_ERR_UNSUPPORTED, "linear %d: in=%lld", k, (long long)d.in);
+        if (!aligned16(d.x) || !aligned16(d.qweight) || (reinterpret_cast<uintptr_t>(d.scales) & 1u) ||
+            (d.zeros && (reinterpret_cast<uintptr_t>(d.zeros) & 3u)) || (d.s16 && !aligned16(d.s16)) ||
+            (reinterpret_cast<uintptr_t>(d.y) & 1u))
+            return fail(AWQ_ERR_ALIGN, "linear %d: misaligned pointer", k);
+        b.lin[k] = awq::DecLinear{d.x, d.qweight, d.scales, d.zeros, d.s16, d.y, d.in, d.out};
+    }
+    int sms;
+    if (awq_status_t s = device_info(&sms)) return s;
+    if (!awq::w4a16_dec_config(b, M, group_size, zeros, sms)) {
+        // outside the one-launch kernel's range (M > 8, or too wide to stage): one by one
+        for (int k = 0; k < n; ++k) {
+            const awq_linear_desc_t &d = descs[k];
+            if (awq_status_t s = awq_linear_w4a16(d.x, M, d.in, d.out, d.qweight, d.scales, d.zeros,
+                                                  d.s16, group_size, d.y, stream))
+                return s;
+        }
+        return AWQ_OK;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    kt_reset(3);
+    kt_begin(3, st);
+    AWQ_CUDA(awq::launch_w4a16_dec(b, static_cast<int>(M), group_size, zeros, st));
+    kt_end(3, st);
+    return AWQ_OK;
+}
+
 awq_status_t awq_fold_scale(const void *P, int p_dtype, int64_t rows, int64_t cols,
                             const uint16_t *s16, void *out, void *stream) {
     g_last_error.clear();
@@ -663,7 +708,8 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (M <= 4) {
-        // decode: CUDA-core kernels streaming the packed weights, one launch
+        // decode: CUDA-core kernels streaming the packed weights (one linear; several
+        // linears at once go through awq_linear_w4a16_batch)
         kt_reset(3);
         kt_begin(3, st);
         AWQ_CUDA(awq::launch_w4a16(x, M, in, out, qweight, scales, zeros, s16, group_size, y, st));

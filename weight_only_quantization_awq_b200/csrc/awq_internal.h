@@ -121,6 +121,37 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             int gs, uint16_t *y, const TcPlan &plan, char *workspace,
                             const TcMaps &maps, cudaStream_t st);
 
+// ---- W4A16 decode (M <= 8) over up to DEC_MAX_LINEARS independent linears in one
+// persistent launch.  The work is cut into units of 16 output rows x 4096 input
+// columns; linear l's units are [ucum[l], ucum[l + 1]), spt[l] per 16-row tile.
+// CTA c takes the whole tiles whose first unit lies in [c U / P, (c + 1) U / P)
+// (U units, P = ctas).  Ring depths and buffer sizes come from w4a16_dec_config.
+constexpr int DEC_MAX_LINEARS = 8;
+constexpr int64_t DEC_MAX_M = 8;
+constexpr int64_t DEC_MAX_SMEM = 227 * 1024;
+struct DecLinear {
+    const uint16_t *x;
+    const uint32_t *qweight;
+    const uint16_t *scales;
+    const uint32_t *zeros;
+    const uint16_t *s16;
+    uint16_t *y;
+    int64_t I, O;
+};
+struct DecBatch {
+    DecLinear lin[DEC_MAX_LINEARS];
+    int64_t ucum[DEC_MAX_LINEARS + 1];
+    int spt[DEC_MAX_LINEARS];
+    int n, ctas;
+    int stages, hbufs, xbufs;     // code ring, tile header and activation buffers
+    int hdr_bytes, xbuf_bytes;    // bytes of one header / activation buffer
+    int64_t smem;                 // dynamic shared memory of the launch
+};
+// Fills the partition and the buffer plan of `b` (lin[] and n set by the caller);
+// false when M or the widest linear does not fit the kernel's shared memory.
+bool w4a16_dec_config(DecBatch &b, int64_t M, int gs, bool zeros, int num_sms);
+cudaError_t launch_w4a16_dec(const DecBatch &b, int M, int gs, bool zeros, cudaStream_t st);
+
 // ---- W4A16 apply for decode-sized M (1..16): xs preparation + warp-level MMA kernel
 constexpr int64_t W4A16_MMA_MAX_M = 16;
 int64_t w4a16_mma_workspace_bytes(int64_t M, int64_t I, int gs);

@@ -36,6 +36,7 @@
 
 #include "awq_internal.h"
 #include "awq_ptx.cuh"
+#include "w4a16_frag.cuh"
 
 namespace awq {
 
@@ -44,8 +45,6 @@ namespace {
 constexpr int MMA_WARPS = 8;
 constexpr int MMA_THREADS = MMA_WARPS * 32;
 constexpr int MMA_AHEAD = 4;          // groups of codes in flight per warp
-
-__device__ __forceinline__ int perm8(int p) { return (p >> 1) + 4 * (p & 1); }   // position -> column
 
 // One warp per (token, group) when gs = 128 (4 columns per lane); 2 or 4
 // (token, group) pairs per warp for gs = 64 or 32, reduced over lane segments.
@@ -73,7 +72,7 @@ __global__ void __launch_bounds__(256) xs_prep_kernel(const uint16_t *__restrict
         if (live) {
             // position p of the group -> column perm8 within its 8-column word
             const int p = sub * 4 + e;
-            const int64_t c = g * GS + (p & ~7) + perm8(p & 7);
+            const int64_t c = g * GS + (p & ~7) + frag_perm8(p & 7);
             const float xv = __uint_as_float(static_cast<uint32_t>(x[m * I + c]) << 16);
             v[e] = s16 ? __fdividef(xv, __half2float(__ushort_as_half(s16[c]))) : xv;
         }
@@ -103,19 +102,6 @@ __global__ void __launch_bounds__(256) xs_prep_kernel(const uint16_t *__restrict
         *reinterpret_cast<uint2 *>(xsp + m * I + g * GS + sub * 4) = make_uint2(h[0], h[1]);
         if (sub == 0) xsm[m * nG + g] = make_float2(ldexpf(1.0f, k), sum);
     }
-}
-
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// (1024 + nibble e, 1024 + nibble e + 4) of a packed word as fp16x2.
-__device__ __forceinline__ uint32_t nib2(uint32_t w, int e) {
-    return ((w >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
 }
 
 template <int GS>
@@ -169,7 +155,7 @@ __global__ void __launch_bounds__(MMA_THREADS) w4a16_mma_kernel(
     const int64_t o0 = static_cast<int64_t>(blockIdx.x) * 16 + gi;
     const int64_t nG = I / GS;
     const int64_t nzw = (nG + 7) / 8;
-    const int64_t my = nG > warp ? (nG - warp + MMA_WARPS - 1) / MMA_WARPS : 0;   // groups of this warp
+    const int my = nG > warp ? static_cast<int>((nG - warp + MMA_WARPS - 1) / MMA_WARPS) : 0;   // groups of this warp
 
     // ---- codes of the first groups: independent of the preceding kernels
     Codes<GS> ring[MMA_AHEAD];
@@ -185,9 +171,9 @@ __global__ void __launch_bounds__(MMA_THREADS) w4a16_mma_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[t][e] = 0.0f;
 
-    for (int64_t it = 0; it < my; ++it) {
-        const int64_t grp = warp + it * MMA_WARPS;
-        const int slot = static_cast<int>(it % MMA_AHEAD);
+    for (int it = 0; it < my; ++it) {
+        const int grp = warp + it * MMA_WARPS;
+        const int slot = it & (MMA_AHEAD - 1);
         Codes<GS> c;
 #pragma unroll
         for (int s = 0; s < MMA_AHEAD; ++s)
@@ -201,16 +187,16 @@ __global__ void __launch_bounds__(MMA_THREADS) w4a16_mma_kernel(
         float d0 = 0.0f, d1 = 0.0f, zb0 = 1032.0f, zb1 = 1032.0f;
         if (o0 < O) {
             d0 = __half2float(__ushort_as_half(__ldg(scales + o0 * nG + grp)));
-            if (ZEROS) zb0 = 1024.0f + static_cast<float>((__ldg(zeros + o0 * nzw + grp / 8) >> (4 * (grp % 8))) & 0xFu);
+            if (ZEROS) zb0 = 1024.0f + static_cast<float>((__ldg(zeros + o0 * nzw + (grp >> 3)) >> (4 * (grp & 7))) & 0xFu);
         }
         if (o0 + 8 < O) {
             d1 = __half2float(__ushort_as_half(__ldg(scales + (o0 + 8) * nG + grp)));
-            if (ZEROS) zb1 = 1024.0f + static_cast<float>((__ldg(zeros + (o0 + 8) * nzw + grp / 8) >> (4 * (grp % 8))) & 0xFu);
+            if (ZEROS) zb1 = 1024.0f + static_cast<float>((__ldg(zeros + (o0 + 8) * nzw + (grp >> 3)) >> (4 * (grp & 7))) & 0xFu);
         }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             // B fragments: token gi + 8 t, this lane's quarter of the group (zero past M)
-            const int64_t mb = gi + 8 * t;
+            const int mb = gi + 8 * t;
             uint32_t b[GS / 8];
             if (mb < M) {
                 const uint32_t *src = reinterpret_cast<const uint32_t *>(xsp + mb * I + grp * GS + j * (GS / 4));
@@ -228,14 +214,14 @@ __global__ void __launch_bounds__(MMA_THREADS) w4a16_mma_kernel(
             for (int w = 0; w < NW; ++w) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const uint32_t a[4] = {nib2(c.r0[w], 2 * h), nib2(c.r1[w], 2 * h),
-                                           nib2(c.r0[w], 2 * h + 1), nib2(c.r1[w], 2 * h + 1)};
-                    mma16816(dacc, a, b[4 * w + 2 * h], b[4 * w + 2 * h + 1]);
+                    const uint32_t a[4] = {frag_nib2(c.r0[w], 2 * h), frag_nib2(c.r1[w], 2 * h),
+                                           frag_nib2(c.r0[w], 2 * h + 1), frag_nib2(c.r1[w], 2 * h + 1)};
+                    frag_mma16816(dacc, a, b[4 * w + 2 * h], b[4 * w + 2 * h + 1]);
                 }
             }
             // tokens 2j, 2j + 1 of this n8 tile: scale 2^k and the sum of xs
             float2 f0 = make_float2(0.0f, 0.0f), f1 = make_float2(0.0f, 0.0f);
-            const int64_t m0 = 8 * t + 2 * j;
+            const int m0 = 8 * t + 2 * j;
             if (m0 < M) f0 = __ldg(xsm + m0 * nG + grp);
             if (m0 + 1 < M) f1 = __ldg(xsm + (m0 + 1) * nG + grp);
             acc[t][0] = __fmaf_rn(d0 * f0.x, __fmaf_rn(-zb0, f0.y, dacc[0]), acc[t][0]);
