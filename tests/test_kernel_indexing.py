@@ -9,8 +9,8 @@ and check the invariants the kernels rely on:
   pointer steps.  Every (row, 32-column chunk) must be loaded exactly once, by
   an in-bounds address equal to the direct index, and the lane's zero nibble
   must be the group's.
-* W4A16 batched decode (csrc/k_w4a16_dec.cu): units of 16 rows x 4096 columns
-  over a list of linears; CTA c owns the 16-row tiles whose first unit is in
+* W4A16 batched decode (csrc/k_w4a16_dec.cu): tiles of 8 rows weighing in / 64
+  units over a list of linears; CTA c owns the tiles whose first unit is in
   [c U / P, (c + 1) U / P).  Every tile must be owned by exactly one CTA, the
   tiles a CTA walks must be consecutive, and no CTA may stream much more than
   its share; the staged activations must land in distinct, in-bounds 16-byte
@@ -201,42 +201,37 @@ def test_search_tmem_and_shared_memory_plan():
         assert 1024 + 6 * x_stage + 3 * a_stage + IS * in_stage + bars * 8 + 16 <= 232448
 
 
-# ---- batched decode: partition of tiles over CTAs, staged activation slots
-DEC_KC = 4096
+# ---- batched decode: CTAs per linear, tiles per CTA, staged activation slots
+DEC_TILE_TARGET = 45056
 
 
-def dec_units(linears):
-    """ucum and stages-per-tile of a list of (out, in) linears."""
-    ucum, spt = [0], []
+def dec_plan(linears, sms, gs=128, zeros=True):
+    """w4a16_dec_config restated: tile heights, CTAs per linear and the tile
+    ranges [t0, t1) of every CTA."""
+    rows, weight, tiles = [], [], []
     for O, I in linears:
-        s = -(-I // DEC_KC)
-        spt.append(s)
-        ucum.append(ucum[-1] + -(-O // 16) * s)
-    return ucum, spt
-
-
-def dec_cta_tiles(ucum, spt, u0, u1):
-    """The kernel's dec_first_tile / dec_next_tile walk, restated."""
-    n = len(spt)
-    l = 0
-    while l + 1 < n and u0 >= ucum[l + 1]:
-        l += 1
-    t = (u0 - ucum[l] + spt[l] - 1) // spt[l]
-    a = ucum[l] + t * spt[l]
-    if a >= ucum[l + 1]:
-        if l + 1 >= n:
-            return []
-        l, t, a = l + 1, 0, ucum[l + 1]
-    out = []
-    while a < u1:
-        out.append((l, t, a))
-        a += spt[l]
-        t += 1
-        if a >= ucum[l + 1]:
-            if l + 1 >= n:
-                break
-            l, t, a = l + 1, 0, ucum[l + 1]
-    return out
+        nG, nzw = I // gs, -(-(I // gs) // 8)
+        R = 8 * max(1, DEC_TILE_TARGET // (4 * I))
+        rows.append(R)
+        weight.append(O * (I // 2 + nG * 2 + (nzw * 4 if zeros else 0)))
+        tiles.append(-(-O // R))
+    total = sum(weight)
+    cnt = [min(max(1, sms * w // total), t) for w, t in zip(weight, tiles)]
+    while sum(cnt) > sms:
+        w = max((l for l in range(len(cnt)) if cnt[l] > 1), key=lambda l: (-weight[l] / cnt[l], -l))
+        cnt[w] -= 1
+    while sum(cnt) < sms:
+        cand = [l for l in range(len(cnt)) if cnt[l] < tiles[l]]
+        if not cand:
+            break
+        w = max(cand, key=lambda l: (weight[l] / cnt[l], -l))
+        cnt[w] += 1
+    ranges = []
+    for l, c in enumerate(cnt):
+        T = tiles[l]
+        for ci in range(c):
+            ranges.append((l, ci * T // c, (ci + 1) * T // c))
+    return rows, weight, tiles, cnt, ranges
 
 
 BLOCK7 = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
@@ -245,29 +240,25 @@ BLOCK7 = [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
 @pytest.mark.parametrize("linears,sms", [
     (BLOCK7, 148), ([(4096, 4096)], 148), ([(12288, 4096), (4096, 4096), (22016, 4096), (4096, 11008)], 148),
     ([(17, 64), (5, 1088), (100, 2048)], 148), ([(16, 64)], 148), ([(4100, 4160)], 7),
-    ([(1, 64)] * 8, 3), ([(33, 3072), (2000, 1024)], 148)])
+    ([(1, 64)] * 8, 8), ([(33, 3072), (2000, 1024)], 148), ([(4096, 4096)] * 8, 148)])
 def test_decode_tiles_owned_once_and_balanced(linears, sms):
-    ucum, spt = dec_units(linears)
-    U = ucum[-1]
-    tiles = sum(-(-O // 16) for O, _ in linears)
-    P = min(sms, tiles)
-    owner = {}
-    biggest = max(spt)
-    for c in range(P):
-        u0, u1 = c * U // P, (c + 1) * U // P
-        walk = dec_cta_tiles(ucum, spt, u0, u1)
-        for k, (l, t, a) in enumerate(walk):
-            assert 0 <= t < -(-linears[l][0] // 16)
-            assert a == ucum[l] + t * spt[l] and u0 <= a < u1
-            assert (l, t) not in owner
-            owner[(l, t)] = c
-            if k:
-                pl, pt, _ = walk[k - 1]
-                assert (l, t) == (pl, pt + 1) or (l == pl + 1 and t == 0)
-        units = sum(spt[l] for l, _, _ in walk)
-        # a CTA streams at most its share plus one tile
-        assert units <= U / P + biggest
-    assert len(owner) == tiles
+    """Every tile of every linear belongs to exactly one CTA, each CTA has at
+    least one tile, no more CTAs than SMs; on the decoder block no CTA streams
+    more than 6% above the mean."""
+    rows, weight, tiles, cnt, ranges = dec_plan(linears, sms)
+    assert len(ranges) <= sms and all(c >= 1 for c in cnt)
+    seen = {}
+    for l, t0, t1 in ranges:
+        assert t1 > t0
+        for t in range(t0, t1):
+            assert (l, t) not in seen
+            seen[(l, t)] = True
+    assert len(seen) == sum(tiles)
+    if linears == BLOCK7:
+        per = [weight[l] * (t1 - t0) / tiles[l] for l, t0, t1 in ranges]
+        assert max(per) <= 1.06 * sum(weight) / len(ranges)
+    # every tile holds at most the larger of 44 KB and one 8-row tile of codes
+    assert all(R * I // 2 <= max(DEC_TILE_TARGET, 4 * I) for (_, I), R in zip(linears, rows))
 
 
 @pytest.mark.parametrize("gs", [32, 64, 128])
@@ -283,23 +274,44 @@ def test_decode_staged_slots_distinct_and_contiguous(gs):
         assert got == [4 * kk + j for j in range(4)]
 
 
+def test_decode_unpacking_identities():
+    """The four masks of a packed word give fp16 (1024 + n_e, 1024 + n_e+4) for
+    e = 0, 2 and (1024 + 16 n_e, 1024 + 16 n_e+4) for e = 1, 3, exactly, for
+    every nibble value."""
+    import numpy as np
+    for n in range(16):
+        for pos in range(8):
+            w = n << (4 * pos)
+            w8 = w >> 8
+            halves = {}
+            for e, (src, mask) in enumerate([(w, 0x000F000F), (w, 0x00F000F0), (w8, 0x000F000F), (w8, 0x00F000F0)]):
+                v = (src & mask) | 0x64006400
+                lo, hi = np.array([v & 0xFFFF, v >> 16], np.uint16).view(np.float16).astype(np.float64)
+                halves[e] = (lo, hi)
+            want = {e: [1024.0, 1024.0] for e in range(4)}
+            e, half = {0: (0, 0), 4: (0, 1), 1: (1, 0), 5: (1, 1), 2: (2, 0), 6: (2, 1), 3: (3, 0), 7: (3, 1)}[pos]
+            want[e][half] += n * (16 if e in (1, 3) else 1)
+            for k in range(4):
+                assert halves[k] == tuple(want[k]), (n, pos, k)
+
+
 def test_decode_shared_memory_plan_fits():
-    """The Llama-7B block linears at M = 1 take the 2-buffer plan with four
-    33 KB stages, at M = 2 a 2-buffer plan still; at M = 8 the 4096-wide linears
-    still fit; an 11008-wide linear at M = 8 does not."""
-    def smem(M, linears, gs, zeros, st, hb, xb):
-        hdr = max(32 * (I // gs) + (64 * -(-(I // gs) // 8) if zeros else 0) for _, I in linears)
-        xbuf = max(M * (I + 32) * 2 + -(-(M * (I // gs) * 8) // 16) * 16 for _, I in linears)
-        hdr, xbuf = -(-hdr // 128) * 128, -(-xbuf // 128) * 128
-        return st * 16 * 2112 + hb * hdr + xb * xbuf + 2 * 8 * 16 * 8 * 4 + (2 * st + 2 * hb + 2 * xb) * 8 + 16
+    """Per linear of the decoder block at M = 1: 16-row tiles of the 4096-wide
+    linears and 8-row tiles of the 11008-wide one, at least four slots (over
+    130 KB of codes in flight per SM); at M = 8 the 4096-wide linears still fit;
+    an 11008-wide linear at M = 8 does not."""
+    FIXED = 256 + 256 + 4 * 8 * 16 * 8 * 4
 
-    def plan(M, linears):
-        for o in ((4, 3, 2), (3, 3, 2), (4, 3, 1), (3, 2, 1), (2, 2, 1)):
-            if smem(M, linears, 128, True, *o) <= 227 * 1024:
-                return o
-        return None
+    def plan(M, I, gs=128, zeros=True):
+        nG, nzw = I // gs, -(-(I // gs) // 8)
+        R = 8 * max(1, DEC_TILE_TARGET // (4 * I))
+        slot = -(-(R * I // 2 + R * nG * 2 + (R * nzw * 4 if zeros else 0)) // 128) * 128
+        xbuf = -(-(M * (I + 32) * 2 + M * nG * 16) // 128) * 128
+        st = min(8, (227 * 1024 - FIXED - xbuf) // slot)
+        assert FIXED + xbuf + st * slot <= 227 * 1024
+        return (R, st, st * R * I // 2) if st >= 2 else None
 
-    assert plan(1, BLOCK7) == (4, 3, 2)
-    assert plan(2, BLOCK7) is not None and plan(2, BLOCK7)[2] == 2
-    assert plan(8, [(4096, 4096)]) is not None
-    assert plan(8, BLOCK7) is None
+    assert plan(1, 4096)[0] == 16 and plan(1, 11008)[0] == 8
+    assert all(plan(1, I)[2] >= 130 * 1024 for I in (4096, 11008))
+    assert plan(8, 4096) is not None
+    assert plan(8, 11008) is None

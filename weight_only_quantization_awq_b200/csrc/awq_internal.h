@@ -122,10 +122,12 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const TcMaps &maps, cudaStream_t st);
 
 // ---- W4A16 decode (M <= 8) over up to DEC_MAX_LINEARS independent linears in one
-// persistent launch.  The work is cut into units of 16 output rows x 4096 input
-// columns; linear l's units are [ucum[l], ucum[l + 1]), spt[l] per 16-row tile.
-// CTA c takes the whole tiles whose first unit lies in [c U / P, (c + 1) U / P)
-// (U units, P = ctas).  Ring depths and buffer sizes come from w4a16_dec_config.
+// persistent launch, one CTA per SM.  Each CTA works on one linear: linear l owns
+// the CTAs [cta0[l], cta0[l + 1]) (their number in proportion to its bytes), and
+// its tiles of rows[l] output rows (a multiple of 8; all input columns) are split
+// into equal contiguous ranges among them.  A CTA's ring holds stages[l] slots of
+// slot_bytes[l]; activations take xbuf_bytes[l].  All sizes come from
+// w4a16_dec_config.
 constexpr int DEC_MAX_LINEARS = 8;
 constexpr int64_t DEC_MAX_M = 8;
 constexpr int64_t DEC_MAX_SMEM = 227 * 1024;
@@ -140,15 +142,17 @@ struct DecLinear {
 };
 struct DecBatch {
     DecLinear lin[DEC_MAX_LINEARS];
-    int64_t ucum[DEC_MAX_LINEARS + 1];
-    int spt[DEC_MAX_LINEARS];
+    int cta0[DEC_MAX_LINEARS + 1];
+    int rows[DEC_MAX_LINEARS];
+    int stages[DEC_MAX_LINEARS];
+    int slot_bytes[DEC_MAX_LINEARS];
+    int xbuf_bytes[DEC_MAX_LINEARS];
     int n, ctas;
-    int stages, hbufs, xbufs;     // code ring, tile header and activation buffers
-    int hdr_bytes, xbuf_bytes;    // bytes of one header / activation buffer
     int64_t smem;                 // dynamic shared memory of the launch
 };
-// Fills the partition and the buffer plan of `b` (lin[] and n set by the caller);
-// false when M or the widest linear does not fit the kernel's shared memory.
+// Fills the CTA split and the buffer plan of `b` (lin[] and n set by the caller);
+// false when M or a linear does not fit the kernel's shared memory, or the
+// linears outnumber the SMs.
 bool w4a16_dec_config(DecBatch &b, int64_t M, int gs, bool zeros, int num_sms);
 cudaError_t launch_w4a16_dec(const DecBatch &b, int M, int gs, bool zeros, cudaStream_t st);
 
