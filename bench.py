@@ -60,6 +60,8 @@ LAUNCHES_PER_STEP = 15
 # (sha256 of csrc/k_search.cu, first 16 hex digits).
 SEARCH_TRAFFIC = {
     2: {"source_sha": "44d2be88c075101e", "bytes": 440555008},
+    # dram__bytes_read.sum 146.27 GB + dram__bytes_write.sum 153.65 MB, one launch at full size
+    4: {"source_sha": "d8f32dc52ada6687", "bytes": 146423650000},
 }
 
 
@@ -648,7 +650,16 @@ def main():
     ap.add_argument("--workload", type=int, choices=sorted(BENCH_WORKLOADS), default=4)
     ap.add_argument("--block-search", dest="block_search", action=argparse.BooleanOptionalAction,
                     default=True, help="also time the Llama-7B block's four joint layers' searches")
+    ap.add_argument("--apply-only", dest="apply_only", type=int, nargs="+", default=None, metavar="M",
+                    help="only time the W4A16 apply over the Llama-7B block at these token counts "
+                         "(a short program to profile the apply kernels under ncu; prints one JSON line)")
     args = ap.parse_args()
+    if args.apply_only:
+        import torch
+        torch.cuda.set_device(0)
+        res = measure_block_apply(torch.device("cuda", 0), ms=tuple(args.apply_only), copies=2, reps=1)
+        print(json.dumps({"w4a16_block": {str(m): v for m, v in res.items()}}), flush=True)
+        return 0
     if args.steps is None:
         args.steps = BENCH_WORKLOADS[args.workload]["steps"]
     if args.warmup < 3:

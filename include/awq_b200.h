@@ -212,8 +212,10 @@ awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in,
  * x : [M, in] bf16 device;  y : [M, out] bf16 device, written.  in <= 49152.
  * Storage arguments as produced by awq_pack_int4.  Asynchronous.
  * Kernels by M: 1..4 a CUDA-core kernel streaming the packed weights (no
- * workspace); 5..16 warp-level tensor-core MMA on the unpacked codes (an x / s
- * workspace); 17 and more tcgen05 tensor-core tiles.
+ * workspace), except 2..4 tokens on layers of at least 2^25 weights, which take
+ * the persistent decode kernel of awq_linear_w4a16_batch; 5..16 warp-level
+ * tensor-core MMA on the unpacked codes (an x / s workspace); 17 and more
+ * tcgen05 tensor-core tiles.
  * Precision: x / s16 is rounded to fp16 after a power-of-two scale per
  * (token, group) (2^-11 relative); for M >= 17 (code - z) * scale is also
  * rounded to fp16 once.  Accumulation in fp32.

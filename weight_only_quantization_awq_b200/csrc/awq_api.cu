@@ -707,6 +707,21 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     int sms;
     if (awq_status_t s = device_info(&sms)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M >= 2 && M <= 4 && out * in >= (int64_t(1) << 25)) {
+        // 2-4 tokens on a large layer: the persistent tensor-core decode kernel
+        // (measured faster there; on smaller layers, or one token, the CUDA-core
+        // kernel below wins by its shorter ramp)
+        awq::DecBatch b{};
+        b.lin[0] = awq::DecLinear{x, qweight, scales, zeros, s16, y, in, out};
+        b.n = 1;
+        if (awq::w4a16_dec_config(b, M, group_size, zeros != nullptr, sms)) {
+            kt_reset(3);
+            kt_begin(3, st);
+            AWQ_CUDA(awq::launch_w4a16_dec(b, static_cast<int>(M), group_size, zeros != nullptr, st));
+            kt_end(3, st);
+            return AWQ_OK;
+        }
+    }
     if (M <= 4) {
         // decode: CUDA-core kernels streaming the packed weights (one linear; several
         // linears at once go through awq_linear_w4a16_batch)
