@@ -50,10 +50,10 @@ BENCH_WORKLOADS = {
     2: {"layer": "attn_proj", "quant": "sym", "rotate": 3, "steps": 100, "rows_per_core": 48},
 }
 
-# Kernels of one step: statistics 2 (partial, final); search 9 (absmax, fp16 copy,
-# scale table 2, group parameters, search, row and block reductions, argmin);
-# packing 3 (scale table 2, pack); apply 1.
-LAUNCHES_PER_STEP = 15
+# Kernels of one step: statistics 2 (partial, final); search 10 (absmax, fp16 copy,
+# scale table 2, group parameters, dW range scale, search, row and block
+# reductions, argmin); packing 3 (scale table 2, pack); apply 1.
+LAUNCHES_PER_STEP = 16
 
 # DRAM bytes (read + write) of one search-kernel launch per workload, from an ncu
 # capture of that launch, valid only for the kernel source it was taken on
