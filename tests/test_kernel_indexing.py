@@ -15,6 +15,10 @@ and check the invariants the kernels rely on:
   tiles a CTA walks must be consecutive, and no CTA may stream much more than
   its share; the staged activations must land in distinct, in-bounds 16-byte
   slots whose four fragment-thread reads of a token are one contiguous span.
+* Tensor-core apply (csrc/k_w4a16_tc.cu): the ring depths and TMEM columns a
+  launch asks for must fit one or two CTAs per SM as intended, and the code
+  chunks (128-byte swizzle) must be read unit by unit, once, without bank
+  conflicts within a quarter warp.
 * Fused search (csrc/k_search.cu): CTA pairs deal work units (grid point, 256-row
   pair tile, 512-token block) round-robin; every (grid point, row, token block)
   partial must be written exactly once.
@@ -315,3 +319,74 @@ def test_decode_shared_memory_plan_fits():
     assert all(plan(1, I)[2] >= 130 * 1024 for I in (4096, 11008))
     assert plan(8, 4096) is not None
     assert plan(8, 11008) is None
+
+
+# ---- tensor-core apply (w4a16_tc_kernel): rings, TMEM columns, code chunk reads
+
+def tc_rings(n_tile):
+    """The launch's ring and TMEM plan for a token tile of n_tile (restated)."""
+    xs_b = n_tile * 128
+    bar_bytes = (2 * 4 + 2 * 8 + 2 * 8 + 2) * 8 + 16
+    two = n_tile <= 64
+    budget = (113 if two else 227) * 1024
+    qs = 3
+    xsn = min(8, (budget - 1024 - bar_bytes - qs * 16384) // xs_b)
+    tmem = 256 if two else 512
+    tcols = 32 if n_tile <= 32 else 64 if n_tile <= 64 else 128 if n_tile <= 128 else 256
+    a_st = min(8, (tmem - tcols) // 32)
+    smem = 1024 + xsn * xs_b + qs * 16384 + bar_bytes
+    smem = max(smem, 80 * 1024) if two else max(smem, 120 * 1024)
+    return dict(two=two, xsn=xsn, qs=qs, tmem=tmem, tcols=tcols, a_st=a_st, smem=smem, xs_b=xs_b)
+
+
+@pytest.mark.parametrize("n_tile", list(range(16, 257, 16)))
+def test_tc_rings_fit_shared_memory_and_tmem(n_tile):
+    p = tc_rings(n_tile)
+    assert p["xsn"] >= 2 and p["a_st"] >= 2
+    assert p["smem"] <= 227 * 1024
+    if p["two"]:
+        # two CTAs per SM: shared memory (plus the 1 KB the driver reserves per CTA)
+        # and TMEM (256 columns each) both fit twice
+        assert 2 * (p["smem"] + 1024) <= 228 * 1024 and 2 * p["tmem"] <= 512
+        assert 3 * (p["smem"] + 1024) > 228 * 1024
+    else:
+        # one CTA per SM: more than half the shared memory, so no second CTA is placed
+        # beside one holding all 512 TMEM columns
+        assert 2 * (p["smem"] + 1024) > 228 * 1024
+    assert p["tcols"] >= n_tile and p["tcols"] + 32 * p["a_st"] <= p["tmem"]
+    # the code ring starts on a 1024-byte boundary (128-byte swizzle atoms), and every
+    # activation stage does too (SW128 operand tiles)
+    assert (p["xsn"] * p["xs_b"]) % 1024 == 0 and p["xs_b"] % 1024 == 0
+
+
+def test_tc_code_chunk_reads_cover_units_once_conflict_free():
+    # TMA's 128-byte swizzle stores logical 16-byte unit u of row r (128-byte rows of a
+    # 1024-aligned tile) at unit u ^ (r % 8); thread (row r, half h) reads slab sub's
+    # unit 2 sub + h there.
+    seen = {}
+    for r in range(128):
+        for sub in range(4):
+            for h in range(2):
+                logical = 2 * sub + h
+                phys = (logical ^ (r & 7)) & 7
+                addr = r * 128 + phys * 16
+                assert 0 <= addr and addr + 16 <= 128 * 128
+                assert (r, phys) not in seen
+                seen[(r, phys)] = logical
+    assert len(seen) == 128 * 8
+    # a quarter warp (8 consecutive lanes = 8 consecutive rows, same sub and half)
+    # reads 8 distinct 16-byte bank groups
+    for r0 in range(0, 128, 8):
+        for sub in range(4):
+            for h in range(2):
+                units = {((2 * sub + h) ^ (r & 7)) & 7 for r in range(r0, r0 + 8)}
+                assert len(units) == 8
+
+
+def test_tc_code_chunk_coordinates_aligned():
+    # chunk c of a split starting at slab kb0 is copied from word column (kb0 + 4 c) * 8:
+    # a multiple of 4 words (16 bytes), as a tiled copy's innermost coordinate must be
+    for kb0 in range(0, 200, 7):
+        for c in range(10):
+            x = (kb0 + 4 * c) * 8
+            assert (x * 4) % 16 == 0

@@ -746,11 +746,12 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     // prefill-sized M: tensor cores
     const awq::TcPlan plan = awq::w4a16_tc_plan(M, in, out, sms);
     Workspace ws(st);
-    if (awq_status_t s = ws.reserve(plan.xs_bytes + plan.part_bytes + plan.counter_bytes)) return s;
-    char *wsp = ws.take<char>(plan.xs_bytes + plan.part_bytes + plan.counter_bytes);
+    const int64_t wbytes = plan.xs_bytes + plan.part_bytes + plan.counter_bytes + plan.kx_bytes;
+    if (awq_status_t s = ws.reserve(wbytes)) return s;
+    char *wsp = ws.take<char>(wbytes);
     awq::TcMaps maps;
     if (awq_status_t s = make_map_2d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, qweight, in / 8, out,
-                                     8, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                                     32, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return s;
     if (awq_status_t s = make_map_2d(&maps.xs, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, wsp, in, M,
                                      awq::SLAB_K, static_cast<uint32_t>(plan.n_tile),

@@ -1,26 +1,36 @@
 // W4A16 linear on the tensor cores, for prefill-sized M (AWQ guide, section 三,
 // QuantLinear.forward: y = (x / s) * dequant(W)^T).
 //
-//   xs_absmax_kernel + xs_perm_kernel: xs = fp16((x / s16) * 2^-k), the power of
-//                   two chosen from max |x / s16| so the largest magnitude lands in
-//                   [2^14, 2^15), with the 8 columns of each packed word stored in
-//                   the order (0,4,1,5,2,6,3,7) (see below); y is scaled back by 2^k.
+//   xs_row_kernel:  one block per token m: xs[m] = fp16((x[m] / s16) * 2^-kx[m]),
+//                   the power of two chosen from max_c |x[m, c] / s16[c]| so the
+//                   token's largest magnitude lands in [2^14, 2^15), with the 8
+//                   columns of each packed word stored in the order
+//                   (0,4,1,5,2,6,3,7) (see below); row m of y is scaled back by 2^kx[m].
 //   w4a16_tc_kernel: one CTA per (128-row tile, token tile of 64, 128 or 256,
 //                   K split); one K split whenever the tiles alone fill half the
 //                   SMs, so most prefill shapes have no split-K partials.
-//     warp 8 (TMA)  streams the packed codes [128 rows x 8 words] and the xs tile
-//                   [N tokens x 64 columns] of each 64-column slab into a ring;
-//     warps 0-7     dequantise: two threads per row (32 columns each); the next
-//                   slab's Delta and z are loaded one slab ahead; a word's nibbles e and e+4 become one
-//                   fp16x2 (1024 + code) with a shift and a LOP3 against the 0x6400
-//                   magic; an exact HSUB2 of (1024 + z) and an HMUL2 by
-//                   Delta * 2^-kd (kd from max Delta, so the products stay normal
-//                   fp16) give the pair's dequantised weights with one rounding,
-//                   written to the 128B-swizzled K-major A tile.  The pair order
+//     warp 8 (TMA)  streams the packed codes, 4 slabs [128 rows x 32 words] per
+//                   copy (128-byte swizzle), into a ring released by the
+//                   dequantising warps;
+//     warp 9 (TMA)  streams the xs tile [N tokens x 64 columns] of each 64-column
+//                   slab into a ring released by the MMA;
+//     warps 0-7     dequantise: warp w owns TMEM lane quadrant w % 4 (lane = row of
+//                   the tile) and column half w / 4 of each slab (32 columns, 4
+//                   packed words); each slab's Delta and zero word are loaded four
+//                   slabs ahead; a word's nibbles e and e+4 become one fp16x2
+//                   (1024 + code) with a shift and a LOP3 against the 0x6400 magic;
+//                   an exact HSUB2 of (1024 + z) and an HMUL2 by Delta * 2^-kd[o]
+//                   (kd[o] from the row's largest |Delta|, so the products stay
+//                   normal fp16) give the pair's dequantised weights with one
+//                   rounding, stored into the slab's A stage in TMEM (tcgen05.st,
+//                   16 columns per thread).  Shared memory carries only the two
+//                   streams: the A operand never passes through it.  The pair order
 //                   (e, e+4) is why xs is permuted the same way: the contraction
-//                   over K is order-independent.  y = accumulator * 2^(kx + kd).
-//     warp 9 (MMA)  one thread issues tcgen05.mma M=128 N=tokens K=16 (fp16 in,
-//                   fp32 accumulate in TMEM).
+//                   over K is order-independent.
+//                   y[m][o] = accumulator * 2^kx[m] * 2^kd[o].
+//     warp 10 (MMA) one thread issues tcgen05.mma M=128 N=tokens K=16 with A from
+//                   TMEM and B (xs) from shared memory, fp16 in, fp32 accumulate in
+//                   TMEM.
 //     warps 0-3     epilogue: tcgen05.ld of the accumulator; with one K split
 //                   y is written directly, otherwise each split adds its fp32
 //                   partial, still unscaled (normal-range values, untouched by the
@@ -38,46 +48,23 @@ namespace awq {
 
 namespace {
 
-constexpr int TC_DQ_WARPS = 8;       // dequantisation warps (2 threads per row)
-constexpr int TC_WARP_TMA = 8;
-constexpr int TC_WARP_MMA = 9;
-constexpr int TC_THREADS = 10 * 32;
+constexpr int TC_DQ_WARPS = 8;                        // dequantisation warps: lane quadrant x column half
+constexpr int TC_PF = 4;                              // group parameters fetched this many slabs ahead
+constexpr int TC_WARP_QTMA = TC_DQ_WARPS;             // loads the packed codes
+constexpr int TC_WARP_XTMA = TC_DQ_WARPS + 1;         // loads the activation tiles
+constexpr int TC_WARP_MMA = TC_DQ_WARPS + 2;
+constexpr int TC_THREADS = (TC_DQ_WARPS + 3) * 32;
 constexpr int TC_TOKENS = 256;       // max tokens per tile (MMA N)
-constexpr int RS = 4;                // input ring stages
-constexpr int AS_MAX = 8;            // A ring stages: as many as shared memory allows, up to 8
-constexpr int Q_BYTES = 128 * 32;    // packed codes of a slab: 128 rows x 8 words
-constexpr int A_BYTES = 128 * 128;   // bf16 A tile of a slab
+constexpr int TC_QC = 4;             // slabs per copy of packed codes (128 bytes of each row)
+constexpr int QC_BYTES = 128 * TC_QC * 32;   // packed codes of a chunk: 128 rows x 32 words
+constexpr int QS_MAX = 4;            // code ring stages
+constexpr int XS_MAX = 8;            // activation ring stages
+constexpr int AS_MAX = 8;            // A stages (TMEM)
+constexpr int A_COLS = SLAB_K / 2;   // TMEM columns of one A stage: 64 fp16 per lane
 
-__device__ __forceinline__ int perm8(int p) { return (p >> 1) + 4 * (p & 1); }   // position -> column
 
-// max |x / s16| into max_bits[0] and max |Delta| into max_bits[2] (bit patterns of
-// non-negative floats order as their values).
-__global__ void __launch_bounds__(256) xs_absmax_kernel(const uint16_t *__restrict__ x,
-                                                        const uint16_t *__restrict__ s16, int64_t M,
-                                                        int64_t I, const uint16_t *__restrict__ scales,
-                                                        int64_t n_scales, unsigned *__restrict__ max_bits) {
-    float m = 0.0f, d = 0.0f;
-    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < M * I; k += step) {
-        const int64_t c = k % I;
-        const float xv = __uint_as_float(static_cast<uint32_t>(x[k]) << 16);
-        m = fmaxf(m, fabsf(s16 ? __fdividef(xv, __half2float(__ushort_as_half(s16[c]))) : xv));
-    }
-    for (int64_t k = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; k < n_scales; k += step)
-        d = fmaxf(d, fabsf(__half2float(__ushort_as_half(scales[k]))));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        d = fmaxf(d, __shfl_xor_sync(0xffffffffu, d, off));
-    }
-    if ((threadIdx.x & 31) == 0) {
-        atomicMax(max_bits, __float_as_uint(m));
-        atomicMax(max_bits + 2, __float_as_uint(d));
-    }
-}
-
-// Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero max),
-// clamped to [-125, 125] so that 2^k and 2^-k stay normal floats.
+// Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero or
+// non-finite max), clamped to [-125, 125] so that 2^k and 2^-k stay normal floats.
 __device__ __forceinline__ int pow2_exp(float mx, int top) {
     if (!(mx > 0.0f) || isinf(mx)) return 0;
     int e;
@@ -86,25 +73,86 @@ __device__ __forceinline__ int pow2_exp(float mx, int top) {
     return k < -125 ? -125 : (k > 125 ? 125 : k);
 }
 
-// words: [0] max |xs| bits, [1] kx, [2] max |Delta| bits, [3] kd.
-__global__ void xs_perm_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ s16,
-                               int64_t M, int64_t I, unsigned *__restrict__ words,
-                               uint16_t *__restrict__ xs) {
-    const int k = pow2_exp(__uint_as_float(words[0]), 15);       // max |xs| -> [2^14, 2^15)
+// x / s16 of the 8 columns of packed word w of one token row (s16 may be null: 1).
+__device__ __forceinline__ void xs_word(const uint4 *__restrict__ xr, const uint4 *__restrict__ sr, int w,
+                                        float (&v)[8]) {
+    const uint4 xv = __ldg(xr + w);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    uint32_t sw[4] = {0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u};
+    if (sr) {
+        const uint4 sv = __ldg(sr + w);
+        sw[0] = sv.x; sw[1] = sv.y; sw[2] = sv.z; sw[3] = sv.w;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xFFFF0000u);
+        const __half2 s2 = *reinterpret_cast<const __half2 *>(&sw[e]);
+        v[2 * e] = sr ? __fdividef(x0, __low2float(s2)) : x0;
+        v[2 * e + 1] = sr ? __fdividef(x1, __high2float(s2)) : x1;
+    }
+}
+
+// Blocks [0, M): one token each (see the header), two passes over the row, the second
+// from cache.  Blocks [M, gridDim.x): kd[o] for the rows of W, one warp per row at a
+// time: from the row's largest |Delta| (fp16 bits of non-negative values order as
+// the values), so that 15 * max |Delta| * 2^-kd < 2^15.
+__global__ void __launch_bounds__(256) xs_row_kernel(const uint16_t *__restrict__ x,
+                                                     const uint16_t *__restrict__ s16, int64_t M,
+                                                     int64_t I, const uint16_t *__restrict__ scales,
+                                                     int64_t O, int nG, uint16_t *__restrict__ xs,
+                                                     float *__restrict__ sx, int *__restrict__ kd) {
+    if (blockIdx.x >= M) {
+        const int64_t nw = (static_cast<int64_t>(gridDim.x) - M) * (blockDim.x >> 5);
+        const int lane = threadIdx.x & 31;
+        for (int64_t o = (static_cast<int64_t>(blockIdx.x) - M) * (blockDim.x >> 5) + (threadIdx.x >> 5); o < O;
+             o += nw) {
+            uint32_t mb = 0u;
+            for (int g = lane; g < nG; g += 32) {
+                const uint32_t b = __ldg(scales + o * nG + g) & 0x7FFFu;
+                mb = b > mb ? b : mb;
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const uint32_t t = __shfl_xor_sync(0xffffffffu, mb, off);
+                mb = t > mb ? t : mb;
+            }
+            if (lane == 0) kd[o] = pow2_exp(__half2float(__ushort_as_half(static_cast<unsigned short>(mb))), 11);
+        }
+        return;
+    }
+    __shared__ float wmax[8];
+    const int64_t m = blockIdx.x;
+    const int wpr = static_cast<int>(I / 8);
+    const uint4 *xr = reinterpret_cast<const uint4 *>(x + m * I);
+    const uint4 *sr = reinterpret_cast<const uint4 *>(s16);
+    float mx = 0.0f;
+    for (int w = threadIdx.x; w < wpr; w += blockDim.x) {
+        float v[8];
+        xs_word(xr, sr, w, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(v[e]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = wmax[0];
+    for (int k = 1; k < static_cast<int>(blockDim.x >> 5); ++k) mx = fmaxf(mx, wmax[k]);
+    const int k = pow2_exp(mx, 15);                   // the token's max |xs| -> [2^14, 2^15)
     const float sc = ldexpf(1.0f, -k);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        words[1] = static_cast<unsigned>(k);
-        words[3] = static_cast<unsigned>(pow2_exp(__uint_as_float(words[2]), 11));   // 15 * max Delta < 2^15
+    uint4 *out = reinterpret_cast<uint4 *>(xs + m * I);
+    for (int w = threadIdx.x; w < wpr; w += blockDim.x) {
+        float v[8];
+        xs_word(xr, sr, w, v);
+        uint32_t h[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                 // position pair (2q, 2q + 1) holds columns (q, q + 4)
+            const __half2 hv = __floats2half2_rn(v[q] * sc, v[q + 4] * sc);
+            h[q] = *reinterpret_cast<const uint32_t *>(&hv);
+        }
+        out[w] = make_uint4(h[0], h[1], h[2], h[3]);
     }
-    const int64_t total = M * I;
-    for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
-         q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t m = q / I, c = q % I;
-        const int64_t src = (c & ~int64_t(7)) + perm8(static_cast<int>(c & 7));
-        const float xv = __uint_as_float(static_cast<uint32_t>(x[m * I + src]) << 16);
-        const float v = s16 ? __fdividef(xv, __half2float(__ushort_as_half(s16[src]))) : xv;
-        xs[q] = __half_as_ushort(__float2half_rn(v * sc));
-    }
+    if (threadIdx.x == 0) sx[m] = ldexpf(1.0f, k);
 }
 
 struct TcArgs {
@@ -113,13 +161,17 @@ struct TcArgs {
     int n_tile;            // tokens per tile (multiple of 16, <= 256)
     int splits;            // K splits
     int slabs_per_split;
-    int as;                // A ring stages
+    int as;                // A stages in TMEM (after the accumulator's columns)
+    int tmem_cols;         // TMEM columns allocated
+    int xs_stages;         // activation ring stages
+    int q_stages;          // code ring stages
     const uint16_t *scales;
     const uint32_t *zeros;
     uint16_t *y;
     float *acc32;          // [M][O] fp32, zeroed (splits > 1)
     unsigned *counter;     // [row tiles * token tiles] (splits > 1), zeroed
-    const unsigned *words; // [1] kx, [3] kd: the accumulator is y * 2^-(kx + kd)
+    const float *sx;       // [M]: token m's xs carries 1 / sx[m] (sx[m] = 2^kx[m])
+    const int *kd;         // [O]: row o's dequantised weights carry 2^-kd[o]
 };
 
 __device__ __forceinline__ uint32_t h2sub(uint32_t a, uint32_t b) {
@@ -136,19 +188,19 @@ __device__ __forceinline__ uint32_t h2pack(float a) {
 }
 
 template <bool ZEROS>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow token tiles
     w4a16_tc_kernel(const __grid_constant__ TcMaps maps, const TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int xs_bytes = a.n_tile * 128;
-    const int in_stage = (Q_BYTES + xs_bytes + 1023) / 1024 * 1024;
-    const int AS = a.as;
-    uint8_t *a_ring = base;                                  // AS x 16 KB (1024-aligned)
-    uint8_t *in_ring = a_ring + AS * A_BYTES;                // RS x (xs tile | codes)
-    uint64_t *bars = reinterpret_cast<uint64_t *>(in_ring + RS * in_stage);
-    uint64_t *in_full = bars, *in_empty = bars + RS;
-    uint64_t *a_full = in_empty + RS, *a_empty = a_full + AS_MAX;
+    const int AS = a.as, XS = a.xs_stages, QS = a.q_stages;
+    uint8_t *x_ring = base;                                  // XS x xs tile (multiples of 2 KB)
+    uint8_t *q_ring = x_ring + XS * xs_bytes;                // QS x codes of TC_QC slabs (1024-aligned)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(q_ring + QS * QC_BYTES);
+    uint64_t *q_full = bars, *q_empty = bars + QS_MAX;
+    uint64_t *x_full = q_empty + QS_MAX, *x_empty = x_full + XS_MAX;
+    uint64_t *a_full = x_empty + XS_MAX, *a_empty = a_full + AS_MAX;
     uint64_t *acc_full = a_empty + AS_MAX, *drain = acc_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -163,12 +215,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int64_t kb0 = static_cast<int64_t>(split) * a.slabs_per_split;
     const int64_t kb1 = kb0 + a.slabs_per_split < nK ? kb0 + a.slabs_per_split : nK;
     const int nslab = static_cast<int>(kb1 > kb0 ? kb1 - kb0 : 0);
+    const int nchunk = (nslab + TC_QC - 1) / TC_QC;
+    // accumulator: columns [0, tcols); A stage s: columns [tcols + 32 s, tcols + 32 s + 32)
     const uint32_t tcols = a.n_tile <= 32 ? 32 : (a.n_tile <= 64 ? 64 : (a.n_tile <= 128 ? 128 : 256));
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < RS; ++s) {
-            mbar_init(&in_full[s], 1);
-            mbar_init(&in_empty[s], TC_DQ_WARPS + 1);   // dequant warps read the codes, the MMA reads xs
+        for (int s = 0; s < QS; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], TC_DQ_WARPS);      // released once the dequantisers read the codes
+        }
+        for (int s = 0; s < XS; ++s) {
+            mbar_init(&x_full[s], 1);
+            mbar_init(&x_empty[s], 1);                // released by the MMA's commit
         }
         for (int s = 0; s < AS; ++s) {
             mbar_init(&a_full[s], TC_DQ_WARPS);
@@ -181,61 +239,74 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         fence_mbar_init();
     }
     if (warp == TC_WARP_MMA) {
-        tmem_alloc(tmem_slot, tcols);
+        tmem_alloc(tmem_slot, static_cast<uint32_t>(a.tmem_cols));
         tmem_relinquish();
     }
-    if (warp == TC_WARP_TMA && lane == 0) {
-        tma_prefetch_desc(&maps.q);
-        tma_prefetch_desc(&maps.xs);
-    }
+    if (warp == TC_WARP_QTMA && lane == 0) tma_prefetch_desc(&maps.q);
+    if (warp == TC_WARP_XTMA && lane == 0) tma_prefetch_desc(&maps.xs);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == TC_WARP_TMA) {
+    if (warp == TC_WARP_QTMA) {
+        // ---- packed codes, TC_QC slabs (128 bytes of each row) per copy
         if (lane == 0) {
-            int64_t last[RS];
-#pragma unroll
-            for (int s = 0; s < RS; ++s) last[s] = -1;
-            for (int i = 0; i < nslab; ++i) {
-                const uint32_t st = i % RS;
-                if (!mbar_wait(&in_empty[st], ((i / RS) & 1u) ^ 1u, abort_flag)) break;
-                uint8_t *dst = in_ring + st * in_stage;
-                const int32_t kb = static_cast<int32_t>(kb0 + i);
-                mbar_arrive_expect_tx(&in_full[st], Q_BYTES + xs_bytes);
-                tma_load_2d(dst, &maps.xs, &in_full[st], kb * SLAB_K, static_cast<int32_t>(mt * a.n_tile));
-                tma_load_2d(dst + xs_bytes, &maps.q, &in_full[st], kb * 8, static_cast<int32_t>(ot * 128));
-#pragma unroll
-                for (int s = 0; s < RS; ++s)
-                    if (s == static_cast<int>(st)) last[s] = i;
+            int issued = 0;
+            for (int c = 0; c < nchunk; ++c, ++issued) {
+                const int st = c % QS;
+                if (!mbar_wait(&q_empty[st], ((c / QS) & 1u) ^ 1u, abort_flag)) break;
+                mbar_arrive_expect_tx(&q_full[st], QC_BYTES);
+                tma_load_2d(q_ring + st * QC_BYTES, &maps.q, &q_full[st],
+                            static_cast<int32_t>((kb0 + c * TC_QC) * 8), static_cast<int32_t>(ot * 128));
             }
-#pragma unroll
-            for (int s = 0; s < RS; ++s)
-                if (last[s] >= 0) mbar_wait_drain(&in_full[s], static_cast<uint32_t>((last[s] / RS) & 1));
+            for (int st = 0; st < QS; ++st)          // wait (bounded) for the copies in flight
+                if (issued > st) mbar_wait_drain(&q_full[st], static_cast<uint32_t>(((issued - 1 - st) / QS) & 1));
+        }
+        __syncwarp();
+    } else if (warp == TC_WARP_XTMA) {
+        // ---- the activation tile of each slab
+        if (lane == 0) {
+            int issued = 0;
+            for (int i = 0; i < nslab; ++i, ++issued) {
+                const int st = i % XS;
+                if (!mbar_wait(&x_empty[st], ((i / XS) & 1u) ^ 1u, abort_flag)) break;
+                mbar_arrive_expect_tx(&x_full[st], xs_bytes);
+                tma_load_2d(x_ring + st * xs_bytes, &maps.xs, &x_full[st], static_cast<int32_t>((kb0 + i) * SLAB_K),
+                            static_cast<int32_t>(mt * a.n_tile));
+            }
+            for (int st = 0; st < XS; ++st)
+                if (issued > st) mbar_wait_drain(&x_full[st], static_cast<uint32_t>(((issued - 1 - st) / XS) & 1));
         }
         __syncwarp();
     } else if (warp == TC_WARP_MMA) {
         if (lane == 0) {
             const uint32_t idesc = idesc_f16_f32(128, a.n_tile, false);
-            const uint32_t a_base = smem_u32(a_ring), in_base = smem_u32(in_ring);
+            const uint32_t a_base = tmem_base + tcols, x_base = smem_u32(x_ring);
             bool ok = true;
+            uint32_t as = 0, as_ph = 0, xs = 0, xs_ph = 0;
             for (int i = 0; i < nslab && ok; ++i) {
-                const uint32_t st = i % RS, as = i % AS;
-                if (!mbar_wait(&a_full[as], (i / AS) & 1u, abort_flag) ||
-                    !mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) {
+                if (!mbar_wait(&a_full[as], as_ph, abort_flag) || !mbar_wait(&x_full[xs], xs_ph, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = a_base + as * A_BYTES;
-                const uint32_t b_addr = in_base + st * in_stage;
+                const uint32_t a_addr = a_base + as * A_COLS;
+                const uint32_t b_addr = x_base + xs * xs_bytes;
 #pragma unroll
                 for (int k = 0; k < SLAB_K / 16; ++k)
-                    umma_f16(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32),
-                             sdesc_kmajor_sw128(b_addr + k * 32), idesc, (i > 0 || k > 0) ? 1u : 0u);
-                umma_commit(&in_empty[st]);
+                    umma_f16_ts(tmem_base, a_addr + k * 8, sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                                (i > 0 || k > 0) ? 1u : 0u);
+                umma_commit(&x_empty[xs]);
                 umma_commit(&a_empty[as]);
+                if (++as == static_cast<uint32_t>(AS)) {
+                    as = 0;
+                    as_ph ^= 1u;
+                }
+                if (++xs == static_cast<uint32_t>(XS)) {
+                    xs = 0;
+                    xs_ph ^= 1u;
+                }
             }
             if (ok) umma_commit(acc_full);
             umma_commit(drain);
@@ -243,68 +314,112 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---- dequantisation: two threads per row, 32 columns (4 packed words) each.
-        const int r = threadIdx.x >> 1, hh = threadIdx.x & 1;
+        // ---- dequantisation: warp w writes TMEM lanes 32 (w % 4) .. + 31 (lane = row of
+        // the tile), column half w / 4 of each slab (32 columns, 4 packed words).
+        const int r = 32 * (warp & 3) + lane, hh = warp >> 2;
+        const uint32_t a_lane = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + tcols + hh * 16;
         const int64_t o = ot * 128 + r;
         const bool row_ok = o < a.O;
-        const int64_t nG = a.I / a.gs, nzw = (nG + 7) / 8;
-        const float dscale = ldexpf(1.0f, -static_cast<int>(a.words[3]));
-        // Delta and (1024 + z) of this thread's group in slab i (fp16x2, exact).
-        auto group_params = [&](int i, uint32_t &d2, uint32_t &z2) {
-            float d = 0.0f, z = 8.0f;
+        const int nG = static_cast<int>(a.I / a.gs), nzw = (nG + 7) / 8;
+        const int lg = a.gs == 32 ? 5 : (a.gs == 64 ? 6 : 7);          // group sizes are powers of two
+        const uint16_t *srow = a.scales + (row_ok ? o : 0) * nG;
+        const uint32_t *zrow = ZEROS ? a.zeros + (row_ok ? o : 0) * nzw : nullptr;
+        const int col0 = static_cast<int>(kb0 * SLAB_K) + hh * 32;      // this thread's first column
+        const float dscale = ldexpf(1.0f, -(row_ok ? __ldg(a.kd + o) : 0));
+        // The raw scale and zero word of this thread's group in slab i, fetched TC_PF
+        // slabs before use into a register ring (the slab loop is unrolled by TC_PF, so
+        // each slot is a fixed register and no load result is touched early).
+        auto fetch = [&](int i, uint32_t &sraw, uint32_t &zraw) {
+            sraw = 0u;
+            zraw = 0x88888888u;
             if (row_ok && i < nslab) {
-                const int64_t g = ((kb0 + i) * SLAB_K + hh * 32) / a.gs;
-                d = __half2float(__ushort_as_half(__ldg(a.scales + o * nG + g)));
-                if (ZEROS) z = static_cast<float>((__ldg(a.zeros + o * nzw + g / 8) >> (4 * (g % 8))) & 0xFu);
+                const int g = (col0 + i * SLAB_K) >> lg;
+                sraw = __ldg(srow + g);
+                if (ZEROS) zraw = __ldg(zrow + (g >> 3));
             }
-            d2 = h2pack(d * dscale);
-            z2 = h2pack(1024.0f + z);
         };
-        uint32_t d_cur, z_cur, d_nxt, z_nxt;
-        group_params(0, d_cur, z_cur);
+        uint32_t rs[TC_PF], rz[TC_PF];
+#pragma unroll
+        for (int u = 0; u < TC_PF; ++u) fetch(u, rs[u], rz[u]);
         bool ok = true;
-        for (int i = 0; i < nslab; ++i) {
-            const uint32_t st = i % RS, as = i % AS;
-            group_params(i + 1, d_nxt, z_nxt);            // one slab ahead
-            if (!mbar_wait(&in_full[st], (i / RS) & 1u, abort_flag)) { ok = false; break; }
-            if (!mbar_wait(&a_empty[as], ((i / AS) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-            const uint4 qw = *reinterpret_cast<const uint4 *>(in_ring + st * in_stage + xs_bytes + r * 32 + hh * 16);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&in_empty[st]);   // codes read (xs is released by the MMA)
-            uint8_t *dst = a_ring + as * A_BYTES;
+        uint32_t as = 0, as_ph = 0;                      // A ring slot of slab i and its phase
+        uint32_t qs = 0, qs_ph = 0;                      // code ring slot of slab i's chunk and its phase
+        for (int i0 = 0; i0 < nslab && ok; i0 += TC_PF) {
+#pragma unroll
+        for (int u = 0; u < TC_PF; ++u) {
+            const int i = i0 + u;
+            if (i >= nslab) break;
+            const int sub = i % TC_QC;                   // slab within its code chunk
+            // Delta * 2^-kd and (1024 + z) as fp16x2; the second is exact: OR-ing z
+            // into the 0x6400 pattern of 1024 gives 1024 + z.
+            const int g = (col0 + i * SLAB_K) >> lg;
+            const uint32_t z = ZEROS ? (rz[u] >> (4 * (g & 7))) & 0xFu : 8u;
+            const uint32_t d_cur = h2pack(__half2float(__ushort_as_half(static_cast<unsigned short>(rs[u]))) * dscale);
+            const uint32_t z_cur = (0x6400u | z) * 0x00010001u;
+            fetch(i + TC_PF, rs[u], rz[u]);
+            // (waits with one outcome per warp: the TMEM stores below are warp-wide)
+            if (sub == 0 && !__all_sync(0xffffffffu, mbar_wait(&q_full[qs], qs_ph, abort_flag))) {
+                ok = false;
+                break;
+            }
+            // the chunk holds 128-byte rows in the 128-byte swizzle: 16-byte unit u of row
+            // r sits at unit u ^ (r % 8), so the 8 rows of a quarter warp hit distinct banks
+            const uint4 qw = *reinterpret_cast<const uint4 *>(
+                q_ring + qs * QC_BYTES + r * 128 + ((((sub * 2 + hh) ^ (r & 7)) & 7) << 4));
             const uint32_t wv[4] = {qw.x, qw.y, qw.z, qw.w};
+            if (sub == TC_QC - 1 || i == nslab - 1) {     // the chunk's codes are all read
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&q_empty[qs]);
+                if (++qs == static_cast<uint32_t>(QS)) {
+                    qs = 0;
+                    qs_ph ^= 1u;
+                }
+            }
+            uint32_t v[16];
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
-                uint32_t v[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd
+                    // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd:
+                    // TMEM column 4 wd + e of the half (K positions 2 e, 2 e + 1 of the word)
                     const uint32_t b = ((wv[wd] >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
-                    v[e] = h2mul(h2sub(b, z_cur), d_cur);
+                    v[4 * wd + e] = h2mul(h2sub(b, z_cur), d_cur);
                 }
-                *reinterpret_cast<uint4 *>(dst + sw128_offset(r, hh * 4 + wd)) = make_uint4(v[0], v[1], v[2], v[3]);
             }
-            fence_proxy_async_smem();
+            // the A stage may be overwritten once the MMAs that read it have completed
+            if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], as_ph ^ 1u, abort_flag))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_st16(a_lane + as * A_COLS, v);
+            tmem_wait_st();
+            // one arrival per warp: the lanes' completed TMEM stores are ordered before
+            // lane 0's arrive by the tcgen05 fence and the warp barrier
+            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_full[as]);
-            d_cur = d_nxt;
-            z_cur = z_nxt;
+            if (++as == static_cast<uint32_t>(AS)) {
+                as = 0;
+                as_ph ^= 1u;
+            }
         }
-        if (warp < 4) {
-        // ---- epilogue (warps 0-3): thread = TMEM lane = row of the tile
-        const int64_t eo = ot * 128 + threadIdx.x;
+        }
+        // ---- epilogue (the 8 dequantising warps): warp w reads TMEM lane quadrant w % 4
+        // (lane = row of the tile) and the 16-column chunks j of the accumulator with
+        // j % 2 = w / 4
+        const int64_t eo = ot * 128 + 32 * (warp & 3) + lane;
         const bool erow_ok = eo < a.O;
-        named_bar_sync(1, 128);
+        // y = accumulator * 2^kx[m] * 2^kd[o], two normal factors (their product can be subnormal)
+        const float ysd = ldexpf(1.0f, erow_ok ? __ldg(a.kd + eo) : 0);
+        named_bar_sync(1, TC_DQ_WARPS * 32);
         const bool got = ok && nslab > 0 && mbar_wait_sleep(acc_full, 0, abort_flag);
         tc_fence_after();
         const int64_t m0 = mt * a.n_tile;
         const int mcount = static_cast<int>(a.M - m0 < a.n_tile ? a.M - m0 : a.n_tile);
-        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-        // y = accumulator * 2^kx * 2^kd, two normal factors (their product can be subnormal)
-        const float ysx = ldexpf(1.0f, static_cast<int>(a.words[1]));
-        const float ysd = ldexpf(1.0f, static_cast<int>(a.words[3]));
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
         if (__all_sync(0xffffffffu, got)) {
-            for (int c = 0; c < a.n_tile; c += 16) {
+            for (int c = 16 * hh; c < a.n_tile; c += 32) {
                 uint32_t rv[16];
                 tmem_ld16_wait(lane_addr + static_cast<uint32_t>(c), rv);
 #pragma unroll
@@ -314,7 +429,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         const float acc = __uint_as_float(rv[k]);
                         if (a.splits == 1) {
                             a.y[(m0 + n) * a.O + eo] =
-                                __bfloat16_as_ushort(__float2bfloat16_rn((acc * ysx) * ysd));
+                                __bfloat16_as_ushort(__float2bfloat16_rn((acc * __ldg(a.sx + m0 + n)) * ysd));
                         } else {
                             // split-K partials meet unscaled: they lie in the normal range,
                             // where the float atomic's flush of subnormals cannot bite
@@ -326,29 +441,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (a.splits > 1) {
             __threadfence();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, TC_DQ_WARPS * 32);
             if (threadIdx.x == 0) {
                 const unsigned prev = atomicAdd(&a.counter[tile], 1u);
                 *is_last = prev == static_cast<unsigned>(a.splits - 1);
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(1, TC_DQ_WARPS * 32);
             if (*is_last) {
                 __threadfence();
                 if (erow_ok) {
-#pragma unroll 8
-                    for (int n = 0; n < mcount; ++n)
-                        a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(
-                            __float2bfloat16_rn((__ldcg(a.acc32 + (m0 + n) * a.O + eo) * ysx) * ysd));
+#pragma unroll 4
+                    for (int n = hh; n < mcount; n += 2)
+                        a.y[(m0 + n) * a.O + eo] = __bfloat16_as_ushort(__float2bfloat16_rn(
+                            (__ldcg(a.acc32 + (m0 + n) * a.O + eo) * __ldg(a.sx + m0 + n)) * ysd));
                 }
             }
-        }
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == TC_WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, tcols);
+        tmem_dealloc(tmem_base, static_cast<uint32_t>(a.tmem_cols));
     }
 }
 
@@ -397,7 +511,8 @@ TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     const int64_t MT = (M + p.n_tile - 1) / p.n_tile;
     p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
     p.part_bytes = p.splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
-    p.counter_bytes = (OT * MT * 4 + 16 + 255) / 256 * 256;   // 4 scale words, tile counters
+    p.counter_bytes = p.splits > 1 ? (OT * MT * 4 + 255) / 256 * 256 : 0;   // tile counters
+    p.kx_bytes = ((M + O) * 4 + 255) / 256 * 256;                    // kx [M], kd [O]
     return p;
 }
 
@@ -408,18 +523,17 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     const int64_t OT = (O + 127) / 128, MT = (M + plan.n_tile - 1) / plan.n_tile;
     uint16_t *xs = reinterpret_cast<uint16_t *>(workspace);
     float *acc32 = plan.splits > 1 ? reinterpret_cast<float *>(workspace + plan.xs_bytes) : nullptr;
-    unsigned *words = reinterpret_cast<unsigned *>(workspace + plan.xs_bytes + plan.part_bytes);
-    unsigned *xw = words;                                       // [4]: max|xs|, kx, max|Delta|, kd
-    unsigned *counter = words + 4;                              // [OT * MT]
-    // one memset zeroes the fp32 accumulator tile (if any), the scale words and the counters
-    cudaError_t e = cudaMemsetAsync(workspace + plan.xs_bytes, 0, plan.part_bytes + plan.counter_bytes, st);
-    if (e != cudaSuccess) return e;
-    int blocks = static_cast<int>((M * I + 255) / 256);
-    if (blocks > 148 * 8) blocks = 148 * 8;
-    xs_absmax_kernel<<<blocks, 256, 0, st>>>(x, s16, M, I, scales, O * (I / gs), xw);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    xs_perm_kernel<<<blocks, 256, 0, st>>>(x, s16, M, I, xw, xs);
+    unsigned *counter = reinterpret_cast<unsigned *>(workspace + plan.xs_bytes + plan.part_bytes);
+    float *sx = reinterpret_cast<float *>(workspace + plan.xs_bytes + plan.part_bytes + plan.counter_bytes);
+    int *kd = reinterpret_cast<int *>(sx + M);
+    cudaError_t e = cudaSuccess;
+    if (plan.splits > 1) {   // the fp32 accumulator tile and the tile counters start at zero
+        e = cudaMemsetAsync(acc32, 0, plan.part_bytes + plan.counter_bytes, st);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t row_blocks = (O + 7) / 8 < 148 ? (O + 7) / 8 : 148;
+    xs_row_kernel<<<static_cast<unsigned>(M + row_blocks), 256, 0, st>>>(x, s16, M, I, scales, O,
+                                                                          static_cast<int>(I / gs), xs, sx, kd);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     TcArgs a;
@@ -435,16 +549,32 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     a.y = y;
     a.acc32 = acc32;
     a.counter = counter;
-    a.words = xw;
-    const int in_stage = (Q_BYTES + plan.n_tile * 128 + 1023) / 1024 * 1024;
-    const int fixed = 1024 + RS * in_stage + (2 * RS + 2 * AS_MAX + 2) * 8 + 16;
-    // Deep enough that dequantisation runs well ahead of the MMA completions, but
-    // keep two CTAs per SM when the token tile is narrow.
-    int as = (113 * 1024 - fixed) / A_BYTES;
-    if (as < 3) as = (227 * 1024 - fixed) / A_BYTES;
-    as = as > AS_MAX ? AS_MAX : (as < 2 ? 2 : as);
+    a.sx = sx;
+    a.kd = kd;
+    // Token tiles of up to 64 keep two CTAs per SM (half the TMEM and 113 KB of shared
+    // memory each); wider ones take the SM (all 512 TMEM columns, more than half the
+    // shared memory, so no second CTA can be placed beside them).
+    const int xs_b = plan.n_tile * 128;
+    const int bar_bytes = (2 * QS_MAX + 2 * XS_MAX + 2 * AS_MAX + 2) * 8 + 16;
+    const bool two = plan.n_tile <= 64;
+    const int budget = (two ? 113 : 227) * 1024;
+    const int qs = 3;
+    int xsn = (budget - 1024 - bar_bytes - qs * QC_BYTES) / xs_b;
+    xsn = xsn > XS_MAX ? XS_MAX : xsn;
+    if (xsn < 2) return cudaErrorInvalidConfiguration;
+    const int tmem_cols = two ? 256 : 512;
+    const int tcols = plan.n_tile <= 32 ? 32 : (plan.n_tile <= 64 ? 64 : (plan.n_tile <= 128 ? 128 : 256));
+    int as = (tmem_cols - tcols) / A_COLS;
+    as = as > AS_MAX ? AS_MAX : as;
     a.as = as;
-    const int smem = fixed + as * A_BYTES;
+    a.tmem_cols = tmem_cols;
+    a.xs_stages = xsn;
+    a.q_stages = qs;
+    int smem = 1024 + xsn * xs_b + qs * QC_BYTES + bar_bytes;
+    // (at least 80 KB: never three CTAs of 256 TMEM columns on one SM; at least
+    // 120 KB: never two of 512)
+    if (two && smem < 80 * 1024) smem = 80 * 1024;
+    if (!two && smem < 120 * 1024) smem = 120 * 1024;
     const unsigned grid = static_cast<unsigned>(OT * MT * plan.splits);
     if (zeros) {
         e = cudaFuncSetAttribute(w4a16_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
