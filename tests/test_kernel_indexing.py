@@ -330,11 +330,11 @@ def tc_rings(n_tile):
     two = n_tile <= 64
     budget = (113 if two else 227) * 1024
     qs = 3
-    xsn = min(8, (budget - 1024 - bar_bytes - qs * 16384) // xs_b)
+    xsn = min(8, (budget - 1024 - bar_bytes - qs * 16384) // (2 * xs_b))   # stages of two slabs
     tmem = 256 if two else 512
     tcols = 32 if n_tile <= 32 else 64 if n_tile <= 64 else 128 if n_tile <= 128 else 256
-    a_st = min(8, (tmem - tcols) // 32)
-    smem = 1024 + xsn * xs_b + qs * 16384 + bar_bytes
+    a_st = min(8, (tmem - tcols) // 64)                                      # 64 columns: two slabs
+    smem = 1024 + xsn * 2 * xs_b + qs * 16384 + bar_bytes
     smem = max(smem, 80 * 1024) if two else max(smem, 120 * 1024)
     return dict(two=two, xsn=xsn, qs=qs, tmem=tmem, tcols=tcols, a_st=a_st, smem=smem, xs_b=xs_b)
 
@@ -353,7 +353,7 @@ def test_tc_rings_fit_shared_memory_and_tmem(n_tile):
         # one CTA per SM: more than half the shared memory, so no second CTA is placed
         # beside one holding all 512 TMEM columns
         assert 2 * (p["smem"] + 1024) > 228 * 1024
-    assert p["tcols"] >= n_tile and p["tcols"] + 32 * p["a_st"] <= p["tmem"]
+    assert p["tcols"] >= n_tile and p["tcols"] + 64 * p["a_st"] <= p["tmem"]
     # the code ring starts on a 1024-byte boundary (128-byte swizzle atoms), and every
     # activation stage does too (SW128 operand tiles)
     assert (p["xsn"] * p["xs_b"]) % 1024 == 0 and p["xs_b"] % 1024 == 0

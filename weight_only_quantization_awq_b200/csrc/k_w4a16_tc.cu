@@ -60,7 +60,8 @@ constexpr int QC_BYTES = 128 * TC_QC * 32;   // packed codes of a chunk: 128 row
 constexpr int QS_MAX = 4;            // code ring stages
 constexpr int XS_MAX = 8;            // activation ring stages
 constexpr int AS_MAX = 8;            // A stages (TMEM)
-constexpr int A_COLS = SLAB_K / 2;   // TMEM columns of one A stage: 64 fp16 per lane
+constexpr int TC_SPS = 2;            // slabs per pipeline step (one handshake per step)
+constexpr int A_COLS = TC_SPS * SLAB_K / 2;   // TMEM columns of one A stage: 128 fp16 per lane
 
 
 // Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero or
@@ -195,8 +196,9 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int xs_bytes = a.n_tile * 128;
     const int AS = a.as, XS = a.xs_stages, QS = a.q_stages;
-    uint8_t *x_ring = base;                                  // XS x xs tile (multiples of 2 KB)
-    uint8_t *q_ring = x_ring + XS * xs_bytes;                // QS x codes of TC_QC slabs (1024-aligned)
+    const int xstage = TC_SPS * xs_bytes;
+    uint8_t *x_ring = base;                                  // XS x TC_SPS xs tiles (multiples of 2 KB)
+    uint8_t *q_ring = x_ring + XS * xstage;                  // QS x codes of TC_QC slabs (1024-aligned)
     uint64_t *bars = reinterpret_cast<uint64_t *>(q_ring + QS * QC_BYTES);
     uint64_t *q_full = bars, *q_empty = bars + QS_MAX;
     uint64_t *x_full = q_empty + QS_MAX, *x_empty = x_full + XS_MAX;
@@ -216,6 +218,7 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
     const int64_t kb1 = kb0 + a.slabs_per_split < nK ? kb0 + a.slabs_per_split : nK;
     const int nslab = static_cast<int>(kb1 > kb0 ? kb1 - kb0 : 0);
     const int nchunk = (nslab + TC_QC - 1) / TC_QC;
+    const int nstep = (nslab + TC_SPS - 1) / TC_SPS;
     // accumulator: columns [0, tcols); A stage s: columns [tcols + 32 s, tcols + 32 s + 32)
     const uint32_t tcols = a.n_tile <= 32 ? 32 : (a.n_tile <= 64 ? 64 : (a.n_tile <= 128 ? 128 : 256));
 
@@ -265,15 +268,17 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
         }
         __syncwarp();
     } else if (warp == TC_WARP_XTMA) {
-        // ---- the activation tile of each slab
+        // ---- the activation tiles of each step's TC_SPS slabs
         if (lane == 0) {
             int issued = 0;
-            for (int i = 0; i < nslab; ++i, ++issued) {
-                const int st = i % XS;
-                if (!mbar_wait(&x_empty[st], ((i / XS) & 1u) ^ 1u, abort_flag)) break;
-                mbar_arrive_expect_tx(&x_full[st], xs_bytes);
-                tma_load_2d(x_ring + st * xs_bytes, &maps.xs, &x_full[st], static_cast<int32_t>((kb0 + i) * SLAB_K),
-                            static_cast<int32_t>(mt * a.n_tile));
+            for (int t = 0; t < nstep; ++t, ++issued) {
+                const int st = t % XS;
+                if (!mbar_wait(&x_empty[st], ((t / XS) & 1u) ^ 1u, abort_flag)) break;
+                const int cnt = nslab - t * TC_SPS < TC_SPS ? nslab - t * TC_SPS : TC_SPS;
+                mbar_arrive_expect_tx(&x_full[st], static_cast<uint32_t>(cnt * xs_bytes));
+                for (int u = 0; u < cnt; ++u)
+                    tma_load_2d(x_ring + st * xstage + u * xs_bytes, &maps.xs, &x_full[st],
+                                static_cast<int32_t>((kb0 + t * TC_SPS + u) * SLAB_K), static_cast<int32_t>(mt * a.n_tile));
             }
             for (int st = 0; st < XS; ++st)
                 if (issued > st) mbar_wait_drain(&x_full[st], static_cast<uint32_t>(((issued - 1 - st) / XS) & 1));
@@ -285,18 +290,21 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
             const uint32_t a_base = tmem_base + tcols, x_base = smem_u32(x_ring);
             bool ok = true;
             uint32_t as = 0, as_ph = 0, xs = 0, xs_ph = 0;
-            for (int i = 0; i < nslab && ok; ++i) {
+            for (int t = 0; t < nstep && ok; ++t) {
                 if (!mbar_wait(&a_full[as], as_ph, abort_flag) || !mbar_wait(&x_full[xs], xs_ph, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = a_base + as * A_COLS;
-                const uint32_t b_addr = x_base + xs * xs_bytes;
+                const int cnt = nslab - t * TC_SPS < TC_SPS ? nslab - t * TC_SPS : TC_SPS;
+                for (int u = 0; u < cnt; ++u) {
+                    const uint32_t a_addr = a_base + as * A_COLS + u * (SLAB_K / 2);
+                    const uint32_t b_addr = x_base + xs * xstage + u * xs_bytes;
 #pragma unroll
-                for (int k = 0; k < SLAB_K / 16; ++k)
-                    umma_f16_ts(tmem_base, a_addr + k * 8, sdesc_kmajor_sw128(b_addr + k * 32), idesc,
-                                (i > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < SLAB_K / 16; ++k)
+                        umma_f16_ts(tmem_base, a_addr + k * 8, sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                                    (t > 0 || u > 0 || k > 0) ? 1u : 0u);
+                }
                 umma_commit(&x_empty[xs]);
                 umma_commit(&a_empty[as]);
                 if (++as == static_cast<uint32_t>(AS)) {
@@ -387,21 +395,26 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
                 }
             }
             // the A stage may be overwritten once the MMAs that read it have completed
-            if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], as_ph ^ 1u, abort_flag))) {
-                ok = false;
-                break;
+            const int us = i % TC_SPS;                   // slab within its step
+            if (us == 0) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], as_ph ^ 1u, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
             }
-            tc_fence_after();
-            tmem_st16(a_lane + as * A_COLS, v);
-            tmem_wait_st();
-            // one arrival per warp: the lanes' completed TMEM stores are ordered before
-            // lane 0's arrive by the tcgen05 fence and the warp barrier
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&a_full[as]);
-            if (++as == static_cast<uint32_t>(AS)) {
-                as = 0;
-                as_ph ^= 1u;
+            tmem_st16(a_lane + as * A_COLS + us * (SLAB_K / 2), v);
+            if (us == TC_SPS - 1 || i == nslab - 1) {
+                tmem_wait_st();
+                // one arrival per warp: the lanes' completed TMEM stores are ordered before
+                // lane 0's arrive by the tcgen05 fence and the warp barrier
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[as]);
+                if (++as == static_cast<uint32_t>(AS)) {
+                    as = 0;
+                    as_ph ^= 1u;
+                }
             }
         }
         }
@@ -512,7 +525,7 @@ TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
     p.part_bytes = p.splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
     p.counter_bytes = p.splits > 1 ? (OT * MT * 4 + 255) / 256 * 256 : 0;   // tile counters
-    p.kx_bytes = ((M + O) * 4 + 255) / 256 * 256;                    // kx [M], kd [O]
+    p.kx_bytes = ((M + O) * 4 + 255) / 256 * 256;                    // sx [M], kd [O]
     return p;
 }
 
@@ -559,7 +572,7 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     const bool two = plan.n_tile <= 64;
     const int budget = (two ? 113 : 227) * 1024;
     const int qs = 3;
-    int xsn = (budget - 1024 - bar_bytes - qs * QC_BYTES) / xs_b;
+    int xsn = (budget - 1024 - bar_bytes - qs * QC_BYTES) / (TC_SPS * xs_b);
     xsn = xsn > XS_MAX ? XS_MAX : xsn;
     if (xsn < 2) return cudaErrorInvalidConfiguration;
     const int tmem_cols = two ? 256 : 512;
@@ -570,7 +583,7 @@ cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
     a.tmem_cols = tmem_cols;
     a.xs_stages = xsn;
     a.q_stages = qs;
-    int smem = 1024 + xsn * xs_b + qs * QC_BYTES + bar_bytes;
+    int smem = 1024 + xsn * TC_SPS * xs_b + qs * QC_BYTES + bar_bytes;
     // (at least 80 KB: never three CTAs of 256 TMEM columns on one SM; at least
     // 120 KB: never two of 512)
     if (two && smem < 80 * 1024) smem = 80 * 1024;
