@@ -349,33 +349,52 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
         uint32_t rs[TC_PF], rz[TC_PF];
 #pragma unroll
         for (int u = 0; u < TC_PF; ++u) fetch(u, rs[u], rz[u]);
+        static_assert(TC_PF % TC_QC == 0 && TC_QC % TC_SPS == 0, "unrolled block = whole code chunks = whole steps");
         bool ok = true;
-        uint32_t as = 0, as_ph = 0;                      // A ring slot of slab i and its phase
-        uint32_t qs = 0, qs_ph = 0;                      // code ring slot of slab i's chunk and its phase
+        uint32_t as = 0, as_ph = 0;                      // A stage of the step and its phase
+        uint32_t qs = 0, qs_ph = 0;                      // code ring slot of the step's chunk and its phase
         for (int i0 = 0; i0 < nslab && ok; i0 += TC_PF) {
 #pragma unroll
-        for (int u = 0; u < TC_PF; ++u) {
-            const int i = i0 + u;
-            if (i >= nslab) break;
-            const int sub = i % TC_QC;                   // slab within its code chunk
-            // Delta * 2^-kd and (1024 + z) as fp16x2; the second is exact: OR-ing z
-            // into the 0x6400 pattern of 1024 gives 1024 + z.
-            const int g = (col0 + i * SLAB_K) >> lg;
-            const uint32_t z = ZEROS ? (rz[u] >> (4 * (g & 7))) & 0xFu : 8u;
-            const uint32_t d_cur = h2pack(__half2float(__ushort_as_half(static_cast<unsigned short>(rs[u]))) * dscale);
-            const uint32_t z_cur = (0x6400u | z) * 0x00010001u;
-            fetch(i + TC_PF, rs[u], rz[u]);
+        for (int s2 = 0; s2 < TC_PF / TC_SPS; ++s2) {
+            const int ib = i0 + s2 * TC_SPS;             // the step's first slab
+            if (ib >= nslab) break;
+            const int cnt = nslab - ib < TC_SPS ? nslab - ib : TC_SPS;
             // (waits with one outcome per warp: the TMEM stores below are warp-wide)
-            if (sub == 0 && !__all_sync(0xffffffffu, mbar_wait(&q_full[qs], qs_ph, abort_flag))) {
+            if ((s2 * TC_SPS) % TC_QC == 0 && !__all_sync(0xffffffffu, mbar_wait(&q_full[qs], qs_ph, abort_flag))) {
                 ok = false;
                 break;
             }
-            // the chunk holds 128-byte rows in the 128-byte swizzle: 16-byte unit u of row
-            // r sits at unit u ^ (r % 8), so the 8 rows of a quarter warp hit distinct banks
-            const uint4 qw = *reinterpret_cast<const uint4 *>(
-                q_ring + qs * QC_BYTES + r * 128 + ((((sub * 2 + hh) ^ (r & 7)) & 7) << 4));
-            const uint32_t wv[4] = {qw.x, qw.y, qw.z, qw.w};
-            if (sub == TC_QC - 1 || i == nslab - 1) {     // the chunk's codes are all read
+            // unpack all slabs of the step before the handshake, so their chains overlap
+            uint32_t v[TC_SPS][16];
+#pragma unroll
+            for (int us = 0; us < TC_SPS; ++us) {
+                const int u = s2 * TC_SPS + us, i = ib + us;
+                // Delta * 2^-kd and (1024 + z) as fp16x2; the second is exact: OR-ing z
+                // into the 0x6400 pattern of 1024 gives 1024 + z.
+                const int g = (col0 + i * SLAB_K) >> lg;
+                const uint32_t z = ZEROS ? (rz[u] >> (4 * (g & 7))) & 0xFu : 8u;
+                const uint32_t d_cur =
+                    h2pack(__half2float(__ushort_as_half(static_cast<unsigned short>(rs[u]))) * dscale);
+                const uint32_t z_cur = (0x6400u | z) * 0x00010001u;
+                fetch(i + TC_PF, rs[u], rz[u]);
+                // the chunk holds 128-byte rows in the 128-byte swizzle: 16-byte unit w of row
+                // r sits at unit w ^ (r % 8), so the 8 rows of a quarter warp hit distinct banks
+                const int sub = u % TC_QC;               // slab within its code chunk
+                const uint4 qw = *reinterpret_cast<const uint4 *>(
+                    q_ring + qs * QC_BYTES + r * 128 + ((((sub * 2 + hh) ^ (r & 7)) & 7) << 4));
+                const uint32_t wv[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+                for (int wd = 0; wd < 4; ++wd) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd:
+                        // TMEM column 4 wd + e of the half (K positions 2 e, 2 e + 1 of the word)
+                        const uint32_t b = ((wv[wd] >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
+                        v[us][4 * wd + e] = h2mul(h2sub(b, z_cur), d_cur);
+                    }
+                }
+            }
+            if (((s2 + 1) * TC_SPS) % TC_QC == 0 || ib + cnt == nslab) {   // the chunk's codes are all read
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&q_empty[qs]);
                 if (++qs == static_cast<uint32_t>(QS)) {
@@ -383,38 +402,24 @@ __global__ void __launch_bounds__(TC_THREADS, 2)   // two CTAs per SM for narrow
                     qs_ph ^= 1u;
                 }
             }
-            uint32_t v[16];
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    // nibbles e and e+4 -> fp16x2 (1024 + code) -> (code - z) * Delta * 2^-kd:
-                    // TMEM column 4 wd + e of the half (K positions 2 e, 2 e + 1 of the word)
-                    const uint32_t b = ((wv[wd] >> (4 * e)) & 0x000F000Fu) | 0x64006400u;
-                    v[4 * wd + e] = h2mul(h2sub(b, z_cur), d_cur);
-                }
-            }
             // the A stage may be overwritten once the MMAs that read it have completed
-            const int us = i % TC_SPS;                   // slab within its step
-            if (us == 0) {
-                if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], as_ph ^ 1u, abort_flag))) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+            if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[as], as_ph ^ 1u, abort_flag))) {
+                ok = false;
+                break;
             }
-            tmem_st16(a_lane + as * A_COLS + us * (SLAB_K / 2), v);
-            if (us == TC_SPS - 1 || i == nslab - 1) {
-                tmem_wait_st();
-                // one arrival per warp: the lanes' completed TMEM stores are ordered before
-                // lane 0's arrive by the tcgen05 fence and the warp barrier
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[as]);
-                if (++as == static_cast<uint32_t>(AS)) {
-                    as = 0;
-                    as_ph ^= 1u;
-                }
+            tc_fence_after();
+#pragma unroll
+            for (int us = 0; us < TC_SPS; ++us)
+                if (us < cnt) tmem_st16(a_lane + as * A_COLS + us * (SLAB_K / 2), v[us]);
+            tmem_wait_st();
+            // one arrival per warp: the lanes' completed TMEM stores are ordered before
+            // lane 0's arrive by the tcgen05 fence and the warp barrier
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (++as == static_cast<uint32_t>(AS)) {
+                as = 0;
+                as_ph ^= 1u;
             }
         }
         }
