@@ -217,10 +217,12 @@ awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in,
  * tensor-core MMA on the unpacked codes (an x / s workspace); 17 and more
  * tcgen05 tensor-core tiles.
  * Precision: x / s16 is rounded to fp16 after a power-of-two scale per
- * (token, group) (2^-11 relative); for M >= 17 (code - z) * scale is also
- * rounded to fp16 once.  Accumulation in fp32.
- * Ordering: the kernels are launched with programmatic stream serialisation,
- * so their blocks may start while the preceding kernel on `stream` is still
+ * (token, group) for M <= 16, per token for M >= 17 (2^-11 relative); for
+ * M >= 17 (code - z) * scale is also rounded to fp16 once, after a power-of-two
+ * scale per output row.  Accumulation in fp32.
+ * Ordering: the streaming (M <= 4), warp-MMA (5..16) and batched decode
+ * kernels are launched with programmatic stream serialisation, so their
+ * blocks may start while the preceding kernel on `stream` is still
  * running; until that kernel has completed they only ask L2 to prefetch
  * their weights (a hint that reads nothing into the SM), and every read of an
  * argument, and the write of y, happens after it.
