@@ -220,7 +220,7 @@ def check_apply(y_gpu: torch.Tensor, y_ref: np.ndarray):
     assert np.all(err <= bound), (err.max(), np.argmax(err - bound))
 
 
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 16, 33, 300])
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 16, 17, 32, 33, 300])
 @pytest.mark.parametrize("O,I,gs,qt", [(200, 384, 128, 0), (96, 512, 64, 1), (130, 256, 32, 1)])
 def test_linear_w4a16_parity(awq, M, O, I, gs, qt):
     W, X = small_layer(O, I, 64, seed=O + M)
