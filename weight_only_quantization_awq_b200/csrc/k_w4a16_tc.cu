@@ -5,7 +5,10 @@
 //                   the power of two chosen from max_c |x[m, c] / s16[c]| so the
 //                   token's largest magnitude lands in [2^14, 2^15), with the 8
 //                   columns of each packed word stored in the order
-//                   (0,4,1,5,2,6,3,7) (see below); row m of y is scaled back by 2^kx[m].
+//                   (0,4,1,5,2,6,3,7) (see below); row m of y is scaled back by
+//                   sx[m] = 2^kx[m].  Further blocks give each weight row o its
+//                   exponent kd[o] (below).  No reduction crosses blocks, so no
+//                   memset or atomic precedes the main kernel.
 //   w4a16_tc_kernel: one CTA per (128-row tile, token tile of 64, 128 or 256,
 //                   K split); one K split whenever the tiles alone fill half the
 //                   SMs, so most prefill shapes have no split-K partials.
@@ -31,13 +34,22 @@
 //     warp 10 (MMA) one thread issues tcgen05.mma M=128 N=tokens K=16 with A from
 //                   TMEM and B (xs) from shared memory, fp16 in, fp32 accumulate in
 //                   TMEM.
-//     warps 0-3     epilogue: tcgen05.ld of the accumulator; with one K split
+//     A pipeline step is two slabs: the dequantising warps unpack both, then hand
+//     them over with one barrier arrival; the MMA releases both with one commit.
+//     warps 0-7     epilogue: tcgen05.ld of the accumulator (two warps per lane
+//                   quadrant, alternate 16-column chunks); with one K split
 //                   y is written directly, otherwise each split adds its fp32
 //                   partial, still unscaled (normal-range values, untouched by the
 //                   atomic's flush of subnormals), into a zeroed fp32 tile with
 //                   red.global.add (the order of those adds across splits is not
 //                   fixed) and the last CTA of the tile (counter) applies the
 //                   power-of-two scales and converts the tile to bf16.
+//
+// Every wait is an mbarrier wait bounded in time: on expiry the CTA raises its abort
+// flag, every role stops waiting, the loaders wait (again bounded) for their copies in
+// flight, the MMA thread for its MMAs, and the CTA frees its TMEM and exits without
+// writing its tile.  A warp's waits have one outcome for the whole warp before its
+// warp-wide TMEM instructions.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -62,7 +74,6 @@ constexpr int XS_MAX = 8;            // activation ring stages
 constexpr int AS_MAX = 8;            // A stages (TMEM)
 constexpr int TC_SPS = 2;            // slabs per pipeline step (one handshake per step)
 constexpr int A_COLS = TC_SPS * SLAB_K / 2;   // TMEM columns of one A stage: 128 fp16 per lane
-
 
 // Power-of-two exponent k with max * 2^-k in [2^(top-1), 2^top) (0 for a zero or
 // non-finite max), clamped to [-125, 125] so that 2^k and 2^-k stay normal floats.
