@@ -15,10 +15,11 @@ and check the invariants the kernels rely on:
   tiles a CTA walks must be consecutive, and no CTA may stream much more than
   its share; the staged activations must land in distinct, in-bounds 16-byte
   slots whose four fragment-thread reads of a token are one contiguous span.
-* Tensor-core apply (csrc/k_w4a16_tc.cu): the ring depths and TMEM columns a
-  launch asks for must fit one or two CTAs per SM as intended, and the code
-  chunks (128-byte swizzle) must be read unit by unit, once, without bank
-  conflicts within a quarter warp.
+* Tensor-core apply (csrc/k_w4a16_tc.cu): the plan's CTAs must cover every
+  (row tile, token tile, slab) exactly once with no empty K split; the ring
+  depths and TMEM columns a launch asks for must fit one or two CTAs per SM as
+  intended; and the code chunks (128-byte swizzle) must be read unit by unit,
+  once, without bank conflicts within a quarter warp.
 * Fused search (csrc/k_search.cu): CTA pairs deal work units (grid point, 256-row
   pair tile, 512-token block) round-robin; every (grid point, row, token block)
   partial must be written exactly once.
@@ -390,3 +391,56 @@ def test_tc_code_chunk_coordinates_aligned():
         for c in range(10):
             x = (kb0 + 4 * c) * 8
             assert (x * 4) % 16 == 0
+
+
+def tc_plan(M, I, O, sms=148):
+    """w4a16_tc_plan restated: token tile, K splits and slabs per split."""
+    OT = -(-O // 128)
+    nK = I // 64
+    best, best_n = 0.0, 0
+    for n in (256, 128, 64):
+        if n > 64 and M <= n // 2:
+            continue
+        tiles = OT * (-(-M // n))
+        if tiles * 2 < sms:
+            continue
+        waves = -(-tiles // sms)
+        cost = waves * n * (1.5 if n == 64 else 1.0)
+        if best_n == 0 or cost < best:
+            best, best_n = cost, n
+    if best_n > 0:
+        n_tile = best_n if best_n < M else -(-M // 16) * 16
+        return n_tile, 1, nK
+    n_tile = 256 if M >= 256 else -(-M // 16) * 16
+    MT = -(-M // n_tile)
+    target = sms if M >= 128 else 2 * sms
+    splits = max(1, target // (OT * MT))
+    splits = min(splits, nK)
+    spl = -(-nK // splits)
+    splits = -(-nK // spl)
+    return n_tile, splits, spl
+
+
+@pytest.mark.parametrize("M", [17, 32, 33, 64, 100, 255, 256, 257, 300, 1024, 4096])
+@pytest.mark.parametrize("O,I", [(96, 64), (200, 384), (4096, 4096), (11008, 4096), (4096, 11008), (520, 1024)])
+def test_tc_plan_covers_every_tile_and_slab_once(M, O, I):
+    # the kernel's decomposition: CTA b -> tile b / splits (row tile tile % OT, token
+    # tile tile / OT), split b % splits covering slabs [split * spl, min(nK, (split+1) spl))
+    n_tile, splits, spl = tc_plan(M, I, O)
+    assert 16 <= n_tile <= 256 and n_tile % 16 == 0
+    OT, MT, nK = -(-O // 128), -(-M // n_tile), I // 64
+    assert MT * n_tile >= M and (MT - 1) * n_tile < M
+    seen = {}
+    for b in range(OT * MT * splits):
+        tile, split = divmod(b, splits)
+        ot, mt = tile % OT, tile // OT
+        k0, k1 = split * spl, min(nK, (split + 1) * spl)
+        assert k0 < k1, "a split with no slabs"
+        for k in range(k0, k1):
+            key = (ot, mt, k)
+            assert key not in seen
+            seen[key] = b
+    assert len(seen) == OT * MT * nK
+    if splits > 1:
+        # K is split only when whole tiles would leave more than half the SMs idle
+        assert all(OT * -(-M // n) * 2 < 148 or (n > 64 and M <= n // 2) for n in (256, 128, 64))
