@@ -197,3 +197,39 @@ def test_linear_batch_rejects_on_host():
     assert f(descs({}, {"y": None}), 2, 1, 128, NULL) == ARG
     assert f(descs({}, {"in_": 100}), 2, 1, 128, NULL) == UNSUP
     assert f(descs({}, {"x": FAKE + 2}), 2, 1, 128, NULL) == ALIGN
+
+
+def test_linear_binding_checks_operand_sizes_before_any_pointer():
+    """The Python binding refuses operands that do not match the packed layout (a short
+    tensor would be read past its end on the GPU), before the library sees a pointer."""
+    import torch
+    M, I, O, gs = 2, 256, 40, 64
+    nG = I // gs
+    x = torch.zeros((M, I), dtype=torch.bfloat16)
+    q = torch.zeros((O, I // 8), dtype=torch.int32)
+    sc = torch.zeros((O, nG), dtype=torch.float16)
+    z = torch.zeros((O, (nG + 7) // 8), dtype=torch.int32)
+    s16 = torch.ones(I, dtype=torch.float16)
+    cases = [
+        (dict(qweight=q[:, :-1]), "qweight"),
+        (dict(qweight=q.to(torch.int16)), "qweight"),
+        (dict(scales=sc[:-1]), "scales"),
+        (dict(scales=sc.float()), "scales"),
+        (dict(zeros=z[:-1]), "zeros"),
+        (dict(s16=s16[:-8]), "s16"),
+        (dict(x=x.float()), "x"),
+        (dict(group_size=96), "group_size"),
+    ]
+    for change, word in cases:
+        args = dict(x=x, qweight=q, scales=sc, zeros=z, s16=s16, group_size=gs)
+        args.update(change)
+        with pytest.raises(ValueError, match=word):
+            awq.awq_linear_w4a16(**args)
+        with pytest.raises(ValueError, match=word):
+            awq.awq_linear_w4a16_batch([(args["x"], args["qweight"], args["scales"], args["zeros"],
+                                         args["s16"])], args["group_size"])
+    # every size right: refused only because the tensors are not on a GPU
+    with pytest.raises(ValueError, match="CUDA"):
+        awq.awq_linear_w4a16(x, q, sc, z, s16, gs)
+    with pytest.raises(ValueError, match="CUDA"):
+        awq.awq_linear_w4a16(x, q, sc, None, None, gs)

@@ -340,18 +340,42 @@ def awq_pack_int4(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float =
             "group_size": group_size}
 
 
+def _w4a16_operands(x, qweight, scales, zeros, s16, group_size: int, name: str = ""):
+    """Check one linear's operands against the packed layout of awq_pack_int4 before any
+    pointer reaches the library (a short tensor would be read past its end): x [M, in]
+    bf16; qweight [out, in/8] of 4-byte words; scales [out, in/gs] of 2-byte values;
+    zeros [out, ceil(in/gs/8)] of 4-byte words or None; s16 [in] of 2-byte values or
+    None; every tensor contiguous, on CUDA and on x's device.  Returns out."""
+    if x.dim() != 2 or x.dtype != torch.bfloat16:
+        raise ValueError(f"{name}x must be a 2-D bfloat16 tensor")
+    inp = x.shape[1]
+    if group_size <= 0 or inp % 8 or inp % group_size:
+        raise ValueError(f"{name}in={inp} must be a multiple of 8 and of group_size {group_size}")
+    if qweight.element_size() != 4 or qweight.dim() != 2 or qweight.shape[1] != inp // 8:
+        raise ValueError(f"{name}qweight must be [out, {inp // 8}] of 4-byte words")
+    out_f = qweight.shape[0]
+    nG = inp // group_size
+    if scales.element_size() != 2 or scales.numel() != out_f * nG:
+        raise ValueError(f"{name}scales must hold {out_f} x {nG} 2-byte values")
+    if zeros is not None and (zeros.element_size() != 4 or zeros.numel() != out_f * ((nG + 7) // 8)):
+        raise ValueError(f"{name}zeros must hold {out_f} x {(nG + 7) // 8} 4-byte words")
+    if s16 is not None and (s16.element_size() != 2 or s16.numel() != inp):
+        raise ValueError(f"{name}s16 must hold {inp} 2-byte values")
+    for t, n in ((x, "x"), (qweight, "qweight"), (scales, "scales"), (zeros, "zeros"), (s16, "s16")):
+        if t is not None:
+            _dev(t, name + n)
+            if t.device != x.device:
+                raise ValueError(f"{name}{n} is on {t.device}, x on {x.device}")
+    return out_f
+
+
 def awq_linear_w4a16(x: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
                      zeros: torch.Tensor | None, s16: torch.Tensor | None, group_size: int = 128,
                      out: torch.Tensor | None = None):
     """y [M, out] bf16 = (x / s16) @ dequant(qweight, scales, zeros)^T for bf16 x [M, in];
     s16=None when x has already been divided by s (awq_fold_scale)."""
-    _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales")
-    if s16 is not None:
-        _dev(s16, "s16")
-    if x.dtype != torch.bfloat16:
-        raise TypeError("x must be bfloat16")
+    out_f = _w4a16_operands(x, qweight, scales, zeros, s16, group_size)
     M, inp = x.shape
-    out_f = qweight.shape[0]
     if out is None:
         out = torch.empty((M, out_f), dtype=torch.bfloat16, device=x.device)
     _out(out, "out", x, torch.bfloat16, M * out_f)
@@ -383,14 +407,9 @@ def awq_linear_w4a16_batch(layers, group_size: int = 128, outs=None):
     descs = (_LinearDesc * len(layers))()
     ys = []
     for k, (x, qweight, scales, zeros, s16) in enumerate(layers):
-        _dev(x, "x"), _dev(qweight, "qweight"), _dev(scales, "scales")
-        if x.dtype != torch.bfloat16 or x.shape[0] != M:
-            raise ValueError("every x must be bfloat16 with the same number of tokens")
-        if zeros is not None:
-            _dev(zeros, "zeros")
-        if s16 is not None:
-            _dev(s16, "s16")
-        out_f = qweight.shape[0]
+        out_f = _w4a16_operands(x, qweight, scales, zeros, s16, group_size, f"layer {k}: ")
+        if x.shape[0] != M or x.device != layers[0][0].device:
+            raise ValueError("every x must have the same number of tokens, on the same device")
         y = outs[k] if outs is not None else torch.empty((M, out_f), dtype=torch.bfloat16,
                                                           device=x.device)
         _out(y, "y", x, torch.bfloat16, M * out_f)
