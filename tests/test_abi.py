@@ -233,3 +233,34 @@ def test_linear_binding_checks_operand_sizes_before_any_pointer():
         awq.awq_linear_w4a16(x, q, sc, z, s16, gs)
     with pytest.raises(ValueError, match="CUDA"):
         awq.awq_linear_w4a16(x, q, sc, None, None, gs)
+
+
+def test_search_and_pack_bindings_check_layer_inputs():
+    """W [out, in], X [N, in] and s_X [in] float32 are checked before any pointer
+    reaches the library (a narrower X, or a shorter or 16-bit s_X, would be read past
+    its end on the GPU)."""
+    import torch
+    W = torch.zeros((32, 128), dtype=torch.bfloat16)
+    X = torch.zeros((64, 128), dtype=torch.bfloat16)
+    sX = torch.ones(128, dtype=torch.float32)
+    calls = [
+        lambda W, X, sX: awq.awq_search_layer(W, X, sX, 64),
+        lambda W, X, sX: awq.awq_search_points(W, X, sX, [0.5], [1.0], 64),
+        lambda W, X, sX: awq.awq_group_clip(W, X, sX, 0.5, [1.0, 0.9], 64),
+        lambda W, X, sX: awq.awq_pack_int4(W, sX, 0.5, 1.0, 64),
+        lambda W, X, sX: awq.awq_pack_quant(W, sX, 0.5, 1.0, 64),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match="sX"):
+            call(W, X, sX.double())
+        with pytest.raises(ValueError, match="sX"):
+            call(W, X, sX.half())
+        with pytest.raises(ValueError, match="sX"):
+            call(W, X, sX[:-4])
+        with pytest.raises(ValueError, match="2-D"):
+            call(W.reshape(-1), X, sX)
+        with pytest.raises(ValueError, match="CUDA"):
+            call(W, X, sX)
+    for call in calls[:3]:
+        with pytest.raises(ValueError, match="input width"):
+            call(W, X[:, :96], sX)

@@ -155,6 +155,25 @@ def _out(t: torch.Tensor, name: str, like: torch.Tensor, dtype: torch.dtype, num
     return t
 
 
+def _layer_inputs(W: torch.Tensor, sX: torch.Tensor, X: torch.Tensor | None = None):
+    """W [out, in] and s_X [in] fp32 (and X [N, in]) on one device, before any pointer
+    reaches the library: a narrower X or a shorter or 16-bit s_X would be read past its
+    end.  Returns (out, in)."""
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [out, in]")
+    out_f, inp = W.shape
+    if sX.dtype != torch.float32 or sX.numel() != inp:
+        raise ValueError(f"sX must be float32 with {inp} elements (one per input channel)")
+    if X is not None and (X.dim() != 2 or X.shape[1] != inp):
+        raise ValueError("W, X and sX disagree on the input width")
+    for t, n in ((W, "W"), (sX, "sX"), (X, "X")):
+        if t is not None:
+            _dev(t, n)
+            if t.device != W.device:
+                raise ValueError(f"{n} is on {t.device}, W on {W.device}")
+    return out_f, inp
+
+
 def awq_act_stats(X: torch.Tensor, clamp_min: float = 1e-4, out: torch.Tensor | None = None):
     """s_X[i] = max(clamp_min, mean_n |X[n, i]|) for X [N, in] (fp32 or bf16)."""
     _dev(X, "X")
@@ -187,11 +206,8 @@ def awq_search_layer(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, group_s
                      loss_row: bool = False):
     """Grid search of one layer.  Returns dict(loss: np.ndarray [G + C] fp64,
     loss_row: tensor [G + C, out] fp32 or None, best_alpha, best_clip)."""
-    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
-    out_f, inp = W.shape
+    out_f, inp = _layer_inputs(W, sX, X)
     N = X.shape[0]
-    if X.shape[1] != inp or sX.numel() != inp:
-        raise ValueError("W, X and sX disagree on the input width")
     a = np.ascontiguousarray(np.asarray(alpha, dtype=np.float64))
     c = np.ascontiguousarray(np.asarray([] if clip is None else clip, dtype=np.float64))
     loss = np.empty(a.size + c.size, np.float64)
@@ -211,11 +227,8 @@ def awq_search_points(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, alpha,
                       group_size: int = 128, w_bit: int = 4, quant="sym", loss_row: bool = False):
     """The loss at each listed (alpha[k], clip[k]) point (a joint grid).  Returns
     dict(loss: np.ndarray [n] fp64, loss_row: tensor [n, out] fp32 or None, best)."""
-    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
-    out_f, inp = W.shape
+    out_f, inp = _layer_inputs(W, sX, X)
     N = X.shape[0]
-    if X.shape[1] != inp or sX.numel() != inp:
-        raise ValueError("W, X and sX disagree on the input width")
     a = np.ascontiguousarray(np.asarray(alpha, dtype=np.float64).ravel())
     c = np.ascontiguousarray(np.asarray(clip, dtype=np.float64).ravel())
     if a.size != c.size:
@@ -237,11 +250,8 @@ def awq_group_clip(W: torch.Tensor, X: torch.Tensor, sX: torch.Tensor, alpha: fl
     """One clip ratio per (row, group) at s = s_X^alpha: the first ratio of
     clip_grid minimising the group's own output error.  Returns dict(clip_idx:
     uint8 [out, in/gs] device, err: fp32 [out, in/gs, n_clip] device or None)."""
-    _dev(W, "W"), _dev(X, "X"), _dev(sX, "sX")
-    out_f, inp = W.shape
+    out_f, inp = _layer_inputs(W, sX, X)
     N = X.shape[0]
-    if X.shape[1] != inp or sX.numel() != inp:
-        raise ValueError("W, X and sX disagree on the input width")
     g = np.ascontiguousarray(np.asarray(clip_grid, dtype=np.float64).ravel())
     nG = inp // group_size
     idx = torch.empty((out_f, nG), dtype=torch.uint8, device=W.device)
@@ -262,8 +272,7 @@ def awq_pack_quant(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float 
     """Packed storage at w_bit 3 or 4, with one clip ratio for the layer or, given
     clip_idx (uint8 [out, in/gs] device) and clip_grid, one per group.  Same
     dict as awq_pack_int4."""
-    _dev(W, "W"), _dev(sX, "sX")
-    out_f, inp = W.shape
+    out_f, inp = _layer_inputs(W, sX)
     q = _quant_code(quant)
     nG = inp // group_size
     dev = W.device
@@ -319,8 +328,7 @@ def awq_pack_int4(W: torch.Tensor, sX: torch.Tensor, alpha: float, clip: float =
     """Packed storage at (alpha, clip): dict(qweight int32 [out, in/8] (u32 bits),
     scales fp16 [out, in/gs], zeros int32 [out, ceil(in/gs/8)] or None,
     s16 fp16 [in], scales_f32 fp32 or None)."""
-    _dev(W, "W"), _dev(sX, "sX")
-    out_f, inp = W.shape
+    out_f, inp = _layer_inputs(W, sX)
     q = _quant_code(quant)
     nG = inp // group_size
     dev = W.device
