@@ -746,7 +746,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
     // prefill-sized M: tensor cores
     const awq::TcPlan plan = awq::w4a16_tc_plan(M, in, out, sms);
     Workspace ws(st);
-    const int64_t wbytes = plan.xs_bytes + plan.part_bytes + plan.counter_bytes + plan.kx_bytes;
+    const int64_t wbytes = plan.xs_bytes + plan.part_bytes + plan.counter_bytes + plan.scale_bytes;
     if (awq_status_t s = ws.reserve(wbytes)) return s;
     char *wsp = ws.take<char>(wbytes);
     awq::TcMaps maps;

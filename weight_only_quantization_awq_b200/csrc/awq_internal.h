@@ -102,7 +102,7 @@ cudaError_t launch_pack(const void *W, bool w_bf16, int64_t O, int64_t I, int gs
                         const float *s, uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
                         uint16_t *s16, float *scales_f32, cudaStream_t st);
 
-// ---- W4A16 apply on the tensor cores (M >= 5)
+// ---- W4A16 apply on the tensor cores (M >= 17)
 struct TcMaps {
     CUtensorMap q;    // qweight [O][I/8] u32, box 32 words (4 slabs) x 128 rows, 128B swizzle
     CUtensorMap xs;   // permuted, power-of-two scaled fp16 x/s [M][I], box 64 x n_tile, 128B swizzle
@@ -111,11 +111,12 @@ struct TcPlan {
     int n_tile;            // tokens per tile (multiple of 16, <= 256)
     int splits;            // K splits
     int slabs_per_split;
-    int64_t xs_bytes, part_bytes, counter_bytes, kx_bytes;   // workspace pieces (256-byte rounded)
+    int64_t xs_bytes, part_bytes, counter_bytes, scale_bytes;   // workspace pieces (256-byte rounded)
 };
 TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms);
 // workspace: xs (plan.xs_bytes), the fp32 split-K accumulator (plan.part_bytes), the
-// tile counters (plan.counter_bytes), then the per-token and per-row exponents (plan.kx_bytes).
+// tile counters (plan.counter_bytes), then the token scales sx [M] fp32 and the row exponents
+// kd [O] int32 (plan.scale_bytes).
 cudaError_t launch_w4a16_tc(const uint16_t *x, int64_t M, int64_t I, int64_t O,
                             const uint16_t *scales, const uint32_t *zeros, const uint16_t *s16,
                             int gs, uint16_t *y, const TcPlan &plan, char *workspace,

@@ -541,7 +541,7 @@ TcPlan w4a16_tc_plan(int64_t M, int64_t I, int64_t O, int num_sms) {
     p.xs_bytes = (M * I * 2 + 255) / 256 * 256;
     p.part_bytes = p.splits > 1 ? (M * O * 4 + 255) / 256 * 256 : 0;
     p.counter_bytes = p.splits > 1 ? (OT * MT * 4 + 255) / 256 * 256 : 0;   // tile counters
-    p.kx_bytes = ((M + O) * 4 + 255) / 256 * 256;                    // sx [M], kd [O]
+    p.scale_bytes = ((M + O) * 4 + 255) / 256 * 256;                    // sx [M], kd [O]
     return p;
 }
 
