@@ -26,8 +26,12 @@
  *   - Arguments are validated on the host before anything is enqueued; an
  *     invalid call returns AWQ_ERR_ARG / AWQ_ERR_ALIGN / AWQ_ERR_UNSUPPORTED
  *     and enqueues nothing.  A failing CUDA call returns AWQ_ERR_CUDA (see
- *     awq_last_error()).  In-kernel waits are bounded; a wait that gives up
- *     is reported as AWQ_ERR_TIMEOUT by the next synchronising entry point.
+ *     awq_last_error()).  In-kernel waits are bounded.  The search entry
+ *     points synchronise and report a wait that gave up as AWQ_ERR_TIMEOUT;
+ *     the W4A16 apply calls return before their kernels run, and a CTA whose
+ *     wait gives up there exits without writing its part of y.
+ *   - Each call is an NVTX range named after the function (visible under a
+ *     profiler; free otherwise).
  *   - Supported: w_bit in {3, 4} (3-bit codes are stored in the same 4-bit
  *     container); group_size in {32, 64, 128}; in % 64 == 0;
  *     in % group_size == 0; any out >= 1 and N >= 1 (tails are masked).

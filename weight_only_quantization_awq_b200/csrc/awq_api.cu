@@ -267,6 +267,7 @@ double awq_last_kernel_ms(int kind) {
 
 awq_status_t awq_act_stats(const void *X, int x_dtype, int64_t N, int64_t in, float clamp_min,
                            float *sX, void *stream) {
+    awq::NvtxRange nvtx_range("awq_act_stats");
     g_last_error.clear();
     if (!X || !sX) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (!valid_dtype(x_dtype)) return fail(AWQ_ERR_ARG, "bad x_dtype %d", x_dtype);
@@ -402,6 +403,7 @@ awq_status_t awq_search_layer(const void *W, int w_dtype, int64_t out, int64_t i
                               int quant, const double *alpha, int n_alpha, const double *clip,
                               int n_clip, double *loss, float *loss_row, int *best_alpha,
                               int *best_clip, void *stream) {
+    awq::NvtxRange nvtx_range("awq_search_layer");
     g_last_error.clear();
     if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
                                              w_bit, quant, loss_row))
@@ -464,6 +466,7 @@ awq_status_t awq_search_points(const void *W, int w_dtype, int64_t out, int64_t 
                                int x_dtype, int64_t N, const float *sX, int group_size, int w_bit,
                                int quant, const double *alpha, const double *clip, int n_points,
                                double *loss, float *loss_row, int *best, void *stream) {
+    awq::NvtxRange nvtx_range("awq_search_points");
     g_last_error.clear();
     if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
                                              w_bit, quant, loss_row))
@@ -515,6 +518,7 @@ awq_status_t awq_pack_quant(const void *W, int w_dtype, int64_t out, int64_t in,
                             const double *clip_grid, int n_clip, int group_size, int w_bit,
                             int quant, uint32_t *qweight, uint16_t *scales, uint32_t *zeros,
                             uint16_t *s16, float *scales_f32, void *stream) {
+    awq::NvtxRange nvtx_range("awq_pack_quant");
     g_last_error.clear();
     if (awq_status_t s = check_layer(W, w_dtype, out, in, group_size, quant)) return s;
     if (w_bit != 3 && w_bit != 4) return fail(AWQ_ERR_UNSUPPORTED, "w_bit %d (3 or 4)", w_bit);
@@ -565,6 +569,7 @@ awq_status_t awq_group_clip(const void *W, int w_dtype, int64_t out, int64_t in,
                             int x_dtype, int64_t N, const float *sX, double alpha, int group_size,
                             int w_bit, int quant, const double *clip_grid, int n_clip,
                             uint8_t *clip_idx, float *err, void *stream) {
+    awq::NvtxRange nvtx_range("awq_group_clip");
     g_last_error.clear();
     if (awq_status_t s = check_search_inputs(W, w_dtype, out, in, X, x_dtype, N, sX, group_size,
                                              w_bit, quant, err))
@@ -603,12 +608,14 @@ awq_status_t awq_pack_int4(const void *W, int w_dtype, int64_t out, int64_t in, 
                            double alpha, double clip, int group_size, int quant, uint32_t *qweight,
                            uint16_t *scales, uint32_t *zeros, uint16_t *s16, float *scales_f32,
                            void *stream) {
+    awq::NvtxRange nvtx_range("awq_pack_int4");
     return awq_pack_quant(W, w_dtype, out, in, sX, alpha, clip, nullptr, nullptr, 0, group_size, 4,
                           quant, qweight, scales, zeros, s16, scales_f32, stream);
 }
 
 awq_status_t awq_linear_w4a16_batch(const awq_linear_desc_t *descs, int n, int64_t M,
                                     int group_size, void *stream) {
+    awq::NvtxRange nvtx_range("awq_linear_w4a16_batch");
     g_last_error.clear();
     if (!descs) return fail(AWQ_ERR_ARG, "NULL descriptor list");
     if (n < 1 || n > AWQ_MAX_BATCH_LINEARS) return fail(AWQ_ERR_ARG, "n=%d not in [1, %d]", n, AWQ_MAX_BATCH_LINEARS);
@@ -654,6 +661,7 @@ awq_status_t awq_linear_w4a16_batch(const awq_linear_desc_t *descs, int n, int64
 
 awq_status_t awq_fold_scale(const void *P, int p_dtype, int64_t rows, int64_t cols,
                             const uint16_t *s16, void *out, void *stream) {
+    awq::NvtxRange nvtx_range("awq_fold_scale");
     g_last_error.clear();
     if (!P || !s16 || !out) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (!valid_dtype(p_dtype)) return fail(AWQ_ERR_ARG, "bad p_dtype %d", p_dtype);
@@ -670,6 +678,7 @@ awq_status_t awq_fold_scale(const void *P, int p_dtype, int64_t rows, int64_t co
 }
 
 awq_status_t awq_wait_selftest(int64_t limit_cycles, int arrive, void *stream) {
+    awq::NvtxRange nvtx_range("awq_wait_selftest");
     g_last_error.clear();
     if (limit_cycles < 1 || limit_cycles > awq::AWQ_DEFAULT_WAIT_CYCLES)
         return fail(AWQ_ERR_ARG, "limit_cycles out of [1, %lld]", (long long)awq::AWQ_DEFAULT_WAIT_CYCLES);
@@ -691,6 +700,7 @@ awq_status_t awq_linear_w4a16(const uint16_t *x, int64_t M, int64_t in, int64_t 
                               const uint32_t *qweight, const uint16_t *scales,
                               const uint32_t *zeros, const uint16_t *s16, int group_size,
                               uint16_t *y, void *stream) {
+    awq::NvtxRange nvtx_range("awq_linear_w4a16");
     g_last_error.clear();
     if (!x || !qweight || !scales || !y) return fail(AWQ_ERR_ARG, "NULL pointer");
     if (M < 1 || in < 1 || out < 1) return fail(AWQ_ERR_ARG, "bad shape");

@@ -4,9 +4,20 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 namespace awq {
+
+// An NVTX range around one C-ABI call, so that each call shows on a profiler's
+// timeline with its kernels under it.  Without a profiler's NVTX injection library
+// the push and pop return at once.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Record the calling host thread's last-error text (read back by awq_last_error()).
 void set_last_error(const char *msg);

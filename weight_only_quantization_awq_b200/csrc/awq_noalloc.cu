@@ -55,6 +55,7 @@ awq_status_t reject(awq_status_t st, const char *msg) {
 
 extern "C" awq_status_t awq_act_stats_noalloc(const void *X, int x_dtype, int64_t N, int64_t in,
                                               float clamp_min, float *sX, void *stream) {
+    awq::NvtxRange nvtx_range("awq_act_stats_noalloc");
     awq::set_last_error("");
     if (!X || !sX) return reject(AWQ_ERR_ARG, "NULL pointer");
     if (x_dtype != AWQ_F32 && x_dtype != AWQ_BF16) return reject(AWQ_ERR_ARG, "bad x_dtype");
