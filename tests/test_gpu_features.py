@@ -2,8 +2,9 @@
 CPU oracle: 3-bit quantisation, the joint (alpha, clip) grid, per-group clip
 packing, layers of very small weights (the power-of-two range scale of dW),
 the fold of 1/s into the previous operator with the apply that skips the
-division, the bounded-wait self-test, and statistics over more token chunks
-than one grid dimension holds.
+division, the bounded-wait self-test, statistics over more token chunks
+than one grid dimension holds, several linears per launch, and outputs written
+in full (NaN-poisoned output buffers).
 
 Bars as in test_gpu_parity: integer results bit-exact, losses within 1e-3
 relative, selected indices equal or a near-tie of the oracle's own losses
@@ -310,3 +311,29 @@ def test_linear_batch_ragged_against_oracle(awq, M, gs, qt, with_s):
     ys = awq.awq_linear_w4a16_batch(layers, gs)
     for y, y_ref in zip(ys, refs):
         check_apply(y, y_ref)
+
+
+# ------------------------------------------------------------------ every output written
+@pytest.mark.parametrize("M", [1, 3, 8, 16, 33, 256])
+def test_apply_writes_every_output(awq, M):
+    """The output buffer is filled with NaN before the call: every element must be
+    overwritten (a tile that a kernel skipped would otherwise keep whatever the
+    allocator handed back, possibly a previous call's correct values).  Ragged rows
+    (300 = 2 x 128 + 44) over several slabs; every kernel by token count, and the
+    batched call for M <= 8."""
+    O, I, gs = 300, 1024, 128
+    W, X = small_layer(O, I, 64, seed=77)
+    pk = oracle.pack_int4(W, oracle.act_stats(X), 0.5, 1.0, gs, oracle.ASYM)
+    x = apply_activations(M, I, seed=5)
+    y_ref = oracle.linear_w4a16(x, pk["qweight"], pk["scales"], pk["zeros"], pk["s16"], gs)
+    args = (dev(x), dev(pk["qweight"]), dev(pk["scales"]).view(torch.float16), dev(pk["zeros"]),
+            dev(pk["s16"]).view(torch.float16))
+    y = torch.full((M, O), float("nan"), dtype=torch.bfloat16, device="cuda")
+    awq.awq_linear_w4a16(*args, gs, out=y)
+    assert bool(torch.isfinite(y).all())
+    check_apply(y, y_ref)
+    if M <= 8:
+        yb = torch.full((M, O), float("nan"), dtype=torch.bfloat16, device="cuda")
+        awq.awq_linear_w4a16_batch([args], gs, outs=[yb])
+        assert bool(torch.isfinite(yb).all())
+        check_apply(yb, y_ref)
